@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark of the fused verify-and-distill step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...     (one process per GPU, NCCL)
+
+One step = one pass of the whole hot path over one batch: the length head (a1), then the fused
+row pass (a2-a5: verification, acceptance, sampling, loss and gradient) over B = 128 sequences,
+k = 16 drafts, V = 151936 (the ragged high-concurrency workload; b_k varies per sequence).  Inputs
+are seeded synthetic bf16 logits resident in HBM; each step reads 1.2 GB of logits, far more
+than the 126 MB L2, so no flush is needed between steps.  The timed region is bracketed by a
+barrier and a device synchronize on both sides and measured with CUDA events on the launching
+stream; with N GPUs every rank runs its own batch (weak scaling) and the step time is the max
+over ranks.  Rank 0 prints one JSON line.
+
+`--impl reference` times the CPU oracle (fp64, all host cores) on a bounded sample of the same
+workload instead and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from speculative_decoding_verify_distill_b200 import api  # noqa: E402
+from speculative_decoding_verify_distill_b200 import parallel  # noqa: E402
+from speculative_decoding_verify_distill_b200 import synthetic as syn  # noqa: E402
+
+WORKLOAD = "ragged_qwen_b128"
+METRIC = "verified draft tokens/s and fused-pass HBM GB/s (% of B200 peak) at B=128,k=16"
+UNIT = "verified draft tokens/s"
+KERNEL_SRC = os.path.join(ROOT, "speculative_decoding_verify_distill_b200", "csrc", "verify_distill.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "row_pass_kernel_ragged_qwen_b128.md")
+
+
+def algorithmic_bytes(bk: np.ndarray, k: int, kt: int, V: int) -> int:
+    """Bytes the row pass must move, each once: a verified row reads D and T and writes the
+    gradient (6V), an unverified row is zero-filled (2V), a bonus row reads T (2V)."""
+    bk = np.asarray(bk, np.int64)
+    per_seq = bk * 6 * V + (k - bk) * 2 * V + (bk < kt) * 2 * V
+    out = int(per_seq.sum())
+    # per-sequence outputs: accept_len, n_emitted, emitted[k+1], bk, loss rows
+    out += len(bk) * 4 * (3 + k + 1 + k)
+    return out
+
+
+def head_bytes(B: int, H: int, M: int) -> int:
+    return 2 * B * H + 2 * M * H + 2 * M + 4 * M + 8 * B
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        if "hbm_gbs" in d:
+            return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_hash() -> str:
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the row pass from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    txt = open(TRAFFIC_FILE).read()
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
+    t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not h or not t or h.group(1) != kernel_hash():
+        return None
+    return float(t.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def build_inputs(w: syn.Workload, seed_offset: int, dev):
+    wr = w.with_(seed=w.seed + seed_offset)
+    D, T = syn.make_logits(wr, pin=True)
+    h, W1, b1, w2, b2 = syn.make_head(wr)
+    host = dict(D=D, T=T, h=h.pin_memory(), W1=W1, b1=b1, w2=w2, b2=b2)
+    devd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+    return wr, host, devd
+
+
+def cpu_oracle_sample(w: syn.Workload, host, n_seqs: int, threads: int):
+    """Times the oracle (a1..a5, fp64) on the first n_seqs sequences; returns (tokens/s, info)."""
+    import oracle
+    oracle.build()
+    oracle.set_threads(threads)
+    seqs = list(range(n_seqs))
+    D, T = host["D"][seqs], host["T"][seqs]
+    h = host["h"][seqs]
+    t0 = time.perf_counter()
+    _, bk, _ = oracle.length_head(h, host["W1"], host["b1"].double().numpy(), host["w2"], host["b2"], w.k)
+    oracle.verify(D, T, None, bk, w.mode, w.tau, w.philox_seed, 0, seq_ids=seqs)
+    oracle.distill(D, T, bk, w.lam, w.clip_c, w.tau, 1.0, want_grad=True)
+    dt = time.perf_counter() - t0
+    return float(bk.sum()) / dt, dict(seconds=dt, verified=int(bk.sum()), seqs=n_seqs)
+
+
+def run_reference(args, info):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    if info.rank != 0:
+        return
+    w = syn.WORKLOADS[WORKLOAD]
+    wr = w.with_()
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    # bounded sample per step: `threads` sequences (one per host core), cycling over the batch,
+    # capped so the whole run stays within a few minutes
+    per_step = max(1, min(threads, w.B))
+    needed = (args.warmup + args.steps) * per_step
+    seqs = [s % w.B for s in range(needed)]
+    uniq = sorted(set(seqs))
+    D, T = syn.make_logits(wr, seqs=uniq)
+    h, W1, b1, w2, b2 = syn.make_head(wr)
+    pos = {s: j for j, s in enumerate(uniq)}
+    oracle.set_threads(threads)
+    times, verified = [], 0
+    for step in range(args.warmup + args.steps):
+        ss = seqs[step * per_step:(step + 1) * per_step]
+        idx = [pos[s] for s in ss]
+        t0 = time.perf_counter()
+        _, bk, _ = oracle.length_head(h[ss], W1, b1.double().numpy(), w2, b2, w.k)
+        oracle.verify(D[idx], T[idx], None, bk, w.mode, w.tau, w.philox_seed, 0, seq_ids=ss)
+        oracle.distill(D[idx], T[idx], bk, w.lam, w.clip_c, w.tau, 1.0, want_grad=True)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            times.append(dt)
+            verified += int(bk.sum())
+    total = sum(times)
+    value = verified / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "k": w.k, "V": w.V, "H": w.H, "M": w.M,
+                   "sample_per_step": "%d sequences" % per_step},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "%d sequences per step (of %d), fp64 oracle a1-a5 with gradient"
+                                   % (per_step, w.B)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--cpu-seqs", type=int, default=0, help="oracle sample size (0 = auto)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    info = parallel.init_from_env("nccl" if torch.cuda.is_available() else "gloo")
+    if args.impl == "reference":
+        run_reference(args, info)
+        if info.world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CUDA path has no CPU fallback)")
+    torch.cuda.set_device(info.local_rank)
+    dev = torch.device("cuda", info.local_rank)
+    w = syn.WORKLOADS[WORKLOAD]
+    wr, host, d = build_inputs(w, parallel.rank_seed(0, info.rank) if info.rank else 0, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    ws = api.Workspace(w.B, w.k, w.kt, w.M, device=dev)
+    bhat = torch.empty(w.B, dtype=torch.float32, device=dev)
+    bk = torch.empty(w.B, dtype=torch.int32, device=dev)
+    # the row pass reads b_k from the head's output buffer in place
+    vd = api.VerifyDistill(d["D"], d["T"], bk_in=bk, mode=w.mode, temperature=w.tau,
+                           seed=w.philox_seed, lam=w.lam, clip_c=w.clip_c, ws=ws)
+    vd.args.bk = api._ptr(bk)
+    vd.bk = bk
+
+    def step_head_into():
+        api.lib().svd_length_head(api._ptr(d["h"]), api._ptr(d["W1"]), api._ptr(d["b1"]),
+                                  api._ptr(d["w2"]), float(d["b2"]), w.B, w.H, w.M, w.k, 1.0,
+                                  api.BK_CEIL, api._ptr(bhat), api._ptr(bk), ws.ptr, ws.nbytes,
+                                  api._stream())
+
+    # ---------------------------------------------------------------- warm-up
+    for _ in range(args.warmup):
+        step_head_into()
+        vd()
+    torch.cuda.synchronize()
+    if api.svd_get_device_error(ws) != 0:
+        raise SystemExit("device error during warm-up")
+    bk_host = bk.cpu().numpy()
+    acc_host = vd.accept_len.cpu().numpy()
+    ne_host = vd.n_emitted.cpu().numpy()
+
+    # ---------------------------------------------------------------- timed region (device)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = None if args.no_clocks else ClockSampler(dev.index if dev.index is not None else 0)
+    if info.world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(K):
+        ev[s][0].record(stream)
+        step_head_into()
+        ev[s][1].record(stream)
+        vd()
+        ev[s][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clock_rec = clocks.stop() if clocks else None
+    if info.world > 1:
+        torch.distributed.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    head_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
+    rows_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
+    ms_per_step = total_ms / K
+    err = api.svd_get_device_error(ws)
+    if err != 0:
+        raise SystemExit("device error in the timed region: %s" % api.STATUS_NAMES.get(err))
+
+    verified = float(bk_host.sum())
+    accepted = float(acc_host.sum())
+    emitted = float(ne_host.sum())
+    loss = float(vd.loss_total.cpu()[0])
+    red = parallel.reduce_metrics(ms_per_step, verified, accepted, emitted, loss, device=dev)
+    value = red["verified"] / (red["ms"] / 1000.0)
+
+    # ---------------------------------------------------------------- roofline of the row pass
+    rows_avg_ms = statistics.mean(rows_ms)
+    alg = algorithmic_bytes(bk_host, w.k, w.kt, w.V)
+    achieved = alg / (rows_avg_ms / 1000.0) / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = recorded_traffic()
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if args.e2e_steps > 0:
+        out_host = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                    for n, t in (("accept_len", vd.accept_len), ("emitted", vd.emitted),
+                                 ("n_emitted", vd.n_emitted), ("loss_total", vd.loss_total),
+                                 ("bk", bk))}
+        h2d = host["D"].numel() * 2 + host["T"].numel() * 2 + host["h"].numel() * 2
+        d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+        if info.world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            d["D"].copy_(host["D"], non_blocking=True)
+            d["T"].copy_(host["T"], non_blocking=True)
+            d["h"].copy_(host["h"], non_blocking=True)
+            step_head_into()
+            vd()
+            for n, t in (("accept_len", vd.accept_len), ("emitted", vd.emitted),
+                         ("n_emitted", vd.n_emitted), ("loss_total", vd.loss_total), ("bk", bk)):
+                out_host[n].copy_(t, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        red_e = parallel.reduce_metrics(e2e_ms, verified, accepted, emitted, loss, device=dev)
+        e2e = {"value": red_e["verified"] / (red_e["ms"] / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # ---------------------------------------------------------------- CPU oracle baseline
+    cpu = None
+    if info.rank == 0 and not args.no_cpu_baseline and info.world == 1:
+        threads = os.cpu_count() or 1
+        nseq = args.cpu_seqs or max(4, min(w.B, 2 * threads))
+        v, extra = cpu_oracle_sample(wr, host, nseq, threads)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": "first %d of %d sequences, fp64 oracle a1-a5 with gradient, %.1f s"
+                         % (nseq, w.B, extra["seconds"])}
+
+    if info.rank == 0:
+        bk_hist = np.bincount(bk_host, minlength=w.k + 1)[1:].tolist()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": red["ms"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": w.B, "k": w.k, "kt": w.kt, "V": w.V, "H": w.H,
+                       "M": w.M, "mode": "greedy", "lambda": w.lam, "clip_c": w.clip_c,
+                       "storage": "bf16 logits / bf16 gradient, fp32 arithmetic",
+                       "l2": "inputs larger than L2 (%.2f GB of logits per step, no flush)"
+                             % ((host["D"].numel() + host["T"].numel()) * 2 / 1e9),
+                       "parallelism": "dp%d (independent batch per GPU)" % info.world},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "row_pass_kernel", "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": alg,
+                         "avg_launch_ms": rows_avg_ms},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 2 * K,
+            "clocks": clock_rec,
+            "accepted_tokens_per_s": red["accepted"] / (red["ms"] / 1000.0),
+            "emitted_tokens_per_s": red["emitted"] / (red["ms"] / 1000.0),
+            "step_hbm_gbs": (alg + head_bytes(w.B, w.H, w.M)) * info.world / (red["ms"] / 1000.0) / 1e9,
+            "length_head_avg_ms": statistics.mean(head_ms),
+            "bk_hist": bk_hist,
+        }
+        print(json.dumps(line), flush=True)
+    if info.world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

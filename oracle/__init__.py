@@ -58,7 +58,7 @@ def _load():
     lib.orc_length_head.argtypes = [P, P, P, P, f64, i32, i32, i32, i32, f64, i32, P, P, P]
     lib.orc_length_head.restype = i32
     lib.orc_row_stats.argtypes = [P, i32, f64, P, P, P]
-    lib.orc_verify.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, f64, u64, u64,
+    lib.orc_verify.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, f64, u64, u64,
                                P, P, P, P, P, P, P, P, P]
     lib.orc_verify.restype = i32
     lib.orc_distill.argtypes = [P, P, P, i32, i32, i32, i32, f64, f64, f64, f64,
@@ -152,8 +152,10 @@ def sample_inverse_cdf(w, u: float):
     return int(tok), float(margin[0])
 
 
-def verify(D, T, draft, bk, mode: int, tau: float = 1.0, seed: int = 0, step: int = 0):
-    """Truncated verification.  D [B,k,V], T [B,kt,V] bf16; bk [B]; draft [B,k] or None.
+def verify(D, T, draft, bk, mode: int, tau: float = 1.0, seed: int = 0, step: int = 0,
+           seq_ids=None):
+    """Truncated verification.  D [B,k,V], T [B,kt,V] bf16; bk [B]; draft [B,k] or None;
+    seq_ids [B] = index of each sequence in its full batch (Philox counter), default 0..B-1.
 
     Returns a dict of numpy arrays: accept_len, emitted, n_emitted and the per-row diagnostics
     row_x, row_y, row_ratio, row_u, row_acc, fix_margin.
@@ -164,13 +166,14 @@ def verify(D, T, draft, bk, mode: int, tau: float = 1.0, seed: int = 0, step: in
     assert Tb.shape[0] == B and Tb.shape[2] == V
     bka = np.ascontiguousarray(np.asarray(bk, dtype=np.int32))
     dr = None if draft is None else np.ascontiguousarray(np.asarray(draft, dtype=np.int32))
+    sid = None if seq_ids is None else np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int32))
     out = dict(
         accept_len=np.zeros(B, np.int32), emitted=np.zeros((B, k + 1), np.int32),
         n_emitted=np.zeros(B, np.int32), row_x=np.zeros((B, k), np.int32),
         row_y=np.zeros((B, kt), np.int32), row_ratio=np.zeros((B, k), np.float64),
         row_u=np.zeros((B, k), np.float64), row_acc=np.zeros((B, k), np.int32),
         fix_margin=np.zeros(B, np.float64))
-    rc = _load().orc_verify(_ptr(Db), _ptr(Tb), _ptr(dr), _ptr(bka), B, k, kt, V, int(mode),
+    rc = _load().orc_verify(_ptr(Db), _ptr(Tb), _ptr(dr), _ptr(bka), _ptr(sid), B, k, kt, V, int(mode),
                             float(tau), int(seed), int(step), _ptr(out["accept_len"]),
                             _ptr(out["emitted"]), _ptr(out["n_emitted"]), _ptr(out["row_x"]),
                             _ptr(out["row_y"]), _ptr(out["row_ratio"]), _ptr(out["row_u"]),

@@ -261,13 +261,16 @@ static int32_t sample_row(const double* Dw /* NULL for bonus */, const double* T
 /*   (verified rows and the bonus row; -1 elsewhere), row_ratio [B,k] p(x)/q(x), row_u [B,k]   */
 /*   accept uniform, row_acc [B,k] decision (-1 = not verified), fix_margin [B] margin of the  */
 /*   correction/bonus sample (+inf if greedy or none).                                         */
+/*   seq_ids [B] (nullable): index of each sequence in its full batch, used as the Philox       */
+/*   sequence counter (default: its position b in this call), so that a subset of a batch     */
+/*   draws the same uniforms as the whole batch.                                               */
 /* Returns 0, 1 on bad arguments, or 2 if a caller token lies outside [0,V).                   */
 /* ------------------------------------------------------------------------------------------ */
 int orc_verify(const uint16_t* D, const uint16_t* T, const int32_t* draft /* nullable */,
-               const int32_t* bk, int B, int k, int kt, int V, int mode, double tau,
-               uint64_t seed, uint64_t step, int32_t* accept_len, int32_t* emitted,
-               int32_t* n_emitted, int32_t* row_x, int32_t* row_y, double* row_ratio,
-               double* row_u, int32_t* row_acc, double* fix_margin) {
+               const int32_t* bk, const int32_t* seq_ids /* nullable */, int B, int k, int kt,
+               int V, int mode, double tau, uint64_t seed, uint64_t step, int32_t* accept_len,
+               int32_t* emitted, int32_t* n_emitted, int32_t* row_x, int32_t* row_y,
+               double* row_ratio, double* row_u, int32_t* row_acc, double* fix_margin) {
     if (k < 1 || k > 64 || (kt != k && kt != k + 1) || V < 1 || B < 0) return 1;
     for (int b = 0; b < B; ++b) if (bk[b] < 1 || bk[b] > k) return 1;
     int bad = 0;
@@ -279,6 +282,7 @@ int orc_verify(const uint16_t* D, const uint16_t* T, const int32_t* draft /* nul
 #pragma omp for schedule(dynamic, 1)
         for (int b = 0; b < B; ++b) {
             int n = bk[b];
+            int sid = seq_ids ? seq_ids[b] : b;
             int a = n;            /* accepted length = first rejected position, else n */
             int32_t x_tok[64];
             for (int i = 0; i < k + 1; ++i) emitted[(size_t)b * (k + 1) + i] = -1;
@@ -305,7 +309,7 @@ int orc_verify(const uint16_t* D, const uint16_t* T, const int32_t* draft /* nul
                     acc = (x == amT);
                 } else {
                     uint32_t w[4];
-                    orc_philox_words(seed, step, b, i, w);
+                    orc_philox_words(seed, step, sid, i, w);
                     double u = uniform24(w[0]);
                     double logp = Tw[x] / tau - lseT;
                     double logq = Dw[x] / tau - lseD;
@@ -341,7 +345,7 @@ int orc_verify(const uint16_t* D, const uint16_t* T, const int32_t* draft /* nul
                 } else {
                     if (residual) widen_row(D + ((size_t)b * k + fix_row) * (size_t)V, V, Dw);
                     uint32_t w[4];
-                    orc_philox_words(seed, step, b, fix_row, w);
+                    orc_philox_words(seed, step, sid, fix_row, w);
                     double margin = INFINITY;
                     tok = sample_row(residual ? Dw : NULL, Tw, V, tau, uniform24(w[1]), scratch,
                                      &margin);

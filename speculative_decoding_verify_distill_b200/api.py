@@ -1,0 +1,293 @@
+"""Python binding of ``libsvd.so`` -- argument marshalling only.
+
+Every entry point has the name of its C function in ``include/svd.h`` and calls it through
+ctypes with device pointers taken from torch tensors and the current CUDA stream.  PyTorch is
+used for device memory and streams only; all arithmetic runs in the CUDA kernels.  There is no
+fallback: if the library is missing or no GPU is present the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsvd.so")
+
+SVD_OK = 0
+STATUS_NAMES = {0: "SVD_OK", 1: "SVD_ERR_INVALID_ARG", 2: "SVD_ERR_ALIGNMENT",
+                3: "SVD_ERR_WORKSPACE", 4: "SVD_ERR_CUDA", 5: "SVD_ERR_TIMEOUT",
+                6: "SVD_ERR_UNSUPPORTED", 7: "SVD_ERR_TOKEN_RANGE"}
+GREEDY, STOCHASTIC = 0, 1
+BK_CEIL, BK_FLOOR = 0, 1
+
+# field order of svd_row_info (8 x 4 bytes)
+ROW_INFO_FIELDS = ("draft_token", "target_argmax", "accepted", "sample_token", "ratio",
+                   "lse_draft", "lse_target", "loss")
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_U64 = ctypes.c_uint64
+_SZ = ctypes.c_size_t
+
+
+class SvdError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__("%s: %s" % (where, STATUS_NAMES.get(code, "status %d" % code)))
+        self.code = code
+
+
+class VerifyDistillArgs(ctypes.Structure):
+    """Mirror of ``svd_verify_distill_args``."""
+    _fields_ = [
+        ("h", _P), ("W1", _P), ("b1", _P), ("w2", _P), ("b2", _F), ("H", _I), ("M", _I),
+        ("gamma", _F), ("rnd", _I), ("bk_in", _P),
+        ("D", _P), ("T", _P), ("draft_tok", _P), ("B", _I), ("k", _I), ("kt", _I), ("V", _I),
+        ("mode", _I), ("temperature", _F), ("seed", _U64), ("step", _U64),
+        ("lambda_", _F), ("clip_c", _F), ("grad_scale", _F), ("dlogits_fp32", _I),
+        ("bhat", _P), ("bk", _P), ("accept_len", _P), ("emitted", _P), ("n_emitted", _P),
+        ("loss_rows", _P), ("loss_total", _P), ("dlogits", _P), ("row_info", _P),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded ``libsvd.so`` with argument types declared (raises if absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libsvd.so is not built (%s); run "
+                           "`python -m speculative_decoding_verify_distill_b200.build`" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    L.svd_workspace_bytes.argtypes = [_I, _I, _I, _I]
+    L.svd_workspace_bytes.restype = _SZ
+    L.svd_workspace_reset.argtypes = [_P, _SZ, _P]
+    L.svd_length_head.argtypes = [_P, _P, _P, _P, _F, _I, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]
+    L.svd_verify.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _U64, _U64, _P, _P, _P, _P,
+                             _P, _SZ, _P]
+    L.svd_distill_loss_grad.argtypes = [_P, _P, _P, _I, _I, _I, _I, _F, _F, _F, _F, _P, _P, _P, _I,
+                                        _P, _SZ, _P]
+    L.svd_verify_distill.argtypes = [ctypes.POINTER(VerifyDistillArgs), _P, _SZ, _P]
+    L.svd_get_device_error.argtypes = [_P, _P]
+    L.svd_status_string.argtypes = [_I]
+    L.svd_status_string.restype = ctypes.c_char_p
+    L.svd_selftest_wait_timeout.argtypes = [_P, _SZ, _U64, _P]
+    for fn in ("svd_workspace_reset", "svd_length_head", "svd_verify", "svd_distill_loss_grad",
+               "svd_verify_distill", "svd_get_device_error", "svd_selftest_wait_timeout"):
+        getattr(L, fn).restype = _I
+    _lib = L
+    return L
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != SVD_OK:
+        raise SvdError(code, where)
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype != torch.bfloat16:
+        raise TypeError("expected bf16 logits / weights, got %s" % t.dtype)
+    return t
+
+
+class Workspace:
+    """Caller-owned scratch for the kernels: zeroed once, reused across calls on one stream."""
+
+    def __init__(self, B: int, k: int, kt: Optional[int] = None, M: int = 0, device=None):
+        kt = k if kt is None else kt
+        n = int(lib().svd_workspace_bytes(B, k, kt, M))
+        self.nbytes = max(n, 256)
+        # torch's caching allocator returns 512-byte aligned blocks
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device or "cuda")
+        assert self.buf.data_ptr() % 256 == 0
+        self.shape = (B, k, kt, M)
+
+    def fits(self, B, k, kt, M=0) -> bool:
+        return int(lib().svd_workspace_bytes(B, k, kt, M)) <= self.nbytes
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+def _ws(ws, B, k, kt, M, device):
+    if ws is None or not ws.fits(B, k, kt, M):
+        ws = Workspace(B, k, kt, M, device=device)
+    return ws
+
+
+def svd_workspace_bytes(B: int, k: int, kt: int, M: int = 0) -> int:
+    return int(lib().svd_workspace_bytes(B, k, kt, M))
+
+
+def svd_get_device_error(ws: Workspace, stream=None) -> int:
+    return int(lib().svd_get_device_error(ws.ptr, _stream(stream)))
+
+
+def svd_status_string(code: int) -> str:
+    return lib().svd_status_string(int(code)).decode()
+
+
+def svd_length_head(h, W1, b1, w2, b2: float, k: int, gamma: float = 1.0, rnd: int = BK_CEIL,
+                    ws: Optional[Workspace] = None, stream=None):
+    """a1: returns (bhat [B] fp32, b_k [B] int32) on h's device."""
+    B, H = h.shape
+    M = W1.shape[0]
+    dev = h.device
+    ws = _ws(ws, B, k, k, M, dev)
+    bhat = torch.empty(B, dtype=torch.float32, device=dev)
+    bk = torch.empty(B, dtype=torch.int32, device=dev)
+    _check(lib().svd_length_head(_ptr(_bits(h)), _ptr(_bits(W1)), _ptr(b1), _ptr(_bits(w2)),
+                                 float(b2), B, H, M, k, float(gamma), int(rnd), _ptr(bhat),
+                                 _ptr(bk), ws.ptr, ws.nbytes, _stream(stream)), "svd_length_head")
+    return bhat, bk
+
+
+def _row_info_tensor(B, kt, dev):
+    return torch.empty((B, kt, 8), dtype=torch.int32, device=dev)
+
+
+def row_info_dict(ri: torch.Tensor) -> dict:
+    """Split a [B, kt, 8] int32 row-info buffer into named fields (ints / floats)."""
+    out = {}
+    for j, name in enumerate(ROW_INFO_FIELDS):
+        col = ri[..., j]
+        out[name] = col if j < 4 else col.view(torch.float32)
+    return out
+
+
+def svd_verify(D, T, draft_tok, bk, mode: int = GREEDY, temperature: float = 1.0, seed: int = 0,
+               step: int = 0, row_info: bool = False, ws: Optional[Workspace] = None, stream=None):
+    """a2-a4: truncated verification.  Returns dict(accept_len, emitted, n_emitted[, row_info])."""
+    B, k, V = D.shape
+    kt = T.shape[1]
+    dev = D.device
+    ws = _ws(ws, B, k, kt, 0, dev)
+    acc = torch.empty(B, dtype=torch.int32, device=dev)
+    emitted = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+    ne = torch.empty(B, dtype=torch.int32, device=dev)
+    ri = _row_info_tensor(B, kt, dev) if row_info else None
+    _check(lib().svd_verify(_ptr(_bits(D)), _ptr(_bits(T)), _ptr(draft_tok), _ptr(bk), B, k, kt, V,
+                            int(mode), float(temperature), int(seed), int(step), _ptr(acc),
+                            _ptr(emitted), _ptr(ne), _ptr(ri), ws.ptr, ws.nbytes, _stream(stream)),
+           "svd_verify")
+    out = dict(accept_len=acc, emitted=emitted, n_emitted=ne)
+    if ri is not None:
+        out["row_info"] = ri
+    return out
+
+
+def svd_distill_loss_grad(D, T, bk, lam: float, clip_c: float, temperature: float = 1.0,
+                          grad_scale: float = 1.0, dlogits_fp32: bool = False,
+                          ws: Optional[Workspace] = None, stream=None, dlogits=None):
+    """a5: returns dict(loss_rows [B,k], loss_total [1], dlogits [B,k,V])."""
+    B, k, V = D.shape
+    kt = T.shape[1]
+    dev = D.device
+    ws = _ws(ws, B, k, kt, 0, dev)
+    loss_rows = torch.empty((B, k), dtype=torch.float32, device=dev)
+    loss_total = torch.empty(1, dtype=torch.float32, device=dev)
+    if dlogits is None:
+        dlogits = torch.empty((B, k, V), dtype=torch.float32 if dlogits_fp32 else torch.bfloat16,
+                              device=dev)
+    _check(lib().svd_distill_loss_grad(_ptr(_bits(D)), _ptr(_bits(T)), _ptr(bk), B, k, kt, V,
+                                       float(lam), float(clip_c), float(temperature),
+                                       float(grad_scale), _ptr(loss_rows), _ptr(loss_total),
+                                       _ptr(dlogits), int(bool(dlogits_fp32)), ws.ptr, ws.nbytes,
+                                       _stream(stream)), "svd_distill_loss_grad")
+    return dict(loss_rows=loss_rows, loss_total=loss_total, dlogits=dlogits)
+
+
+class VerifyDistill:
+    """Preallocated outputs + argument block for repeated fused calls (the benchmark path)."""
+
+    def __init__(self, D, T, *, head=None, bk_in=None, draft_tok=None, mode=GREEDY,
+                 temperature=1.0, seed=0, step=0, lam=0.5, clip_c=1.0, grad_scale=1.0,
+                 gamma=1.0, rnd=BK_CEIL, dlogits_fp32=False, row_info=False, ws=None):
+        B, k, V = D.shape
+        kt = T.shape[1]
+        dev = D.device
+        self.D, self.T, self.head, self.draft_tok, self.bk_in = D, T, head, draft_tok, bk_in
+        M = head[1].shape[0] if head is not None else 0
+        self.ws = _ws(ws, B, k, kt, M, dev)
+        self.bhat = torch.empty(B, dtype=torch.float32, device=dev)
+        self.bk = torch.empty(B, dtype=torch.int32, device=dev)
+        self.accept_len = torch.empty(B, dtype=torch.int32, device=dev)
+        self.emitted = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+        self.n_emitted = torch.empty(B, dtype=torch.int32, device=dev)
+        self.loss_rows = torch.empty((B, k), dtype=torch.float32, device=dev)
+        self.loss_total = torch.empty(1, dtype=torch.float32, device=dev)
+        self.dlogits = torch.empty((B, k, V), dtype=torch.float32 if dlogits_fp32 else torch.bfloat16,
+                                   device=dev)
+        self.row_info = _row_info_tensor(B, kt, dev) if row_info else None
+        a = VerifyDistillArgs()
+        if head is not None:
+            h, W1, b1, w2, b2 = head
+            a.h, a.W1, a.b1, a.w2 = _ptr(_bits(h)), _ptr(_bits(W1)), _ptr(b1), _ptr(_bits(w2))
+            a.b2, a.H, a.M = float(b2), h.shape[1], W1.shape[0]
+        else:
+            if bk_in is None:
+                raise ValueError("either head or bk_in is required")
+            a.bk_in = _ptr(bk_in)
+        a.gamma, a.rnd = float(gamma), int(rnd)
+        a.D, a.T, a.draft_tok = _ptr(_bits(D)), _ptr(_bits(T)), _ptr(draft_tok)
+        a.B, a.k, a.kt, a.V = B, k, kt, V
+        a.mode, a.temperature, a.seed, a.step = int(mode), float(temperature), int(seed), int(step)
+        a.lambda_, a.clip_c, a.grad_scale = float(lam), float(clip_c), float(grad_scale)
+        a.dlogits_fp32 = int(bool(dlogits_fp32))
+        a.bhat, a.bk = _ptr(self.bhat), _ptr(self.bk)
+        a.accept_len, a.emitted, a.n_emitted = _ptr(self.accept_len), _ptr(self.emitted), _ptr(self.n_emitted)
+        a.loss_rows, a.loss_total, a.dlogits = _ptr(self.loss_rows), _ptr(self.loss_total), _ptr(self.dlogits)
+        a.row_info = _ptr(self.row_info)
+        self.args = a
+
+    def set_step(self, step: int):
+        self.args.step = int(step)
+
+    def __call__(self, stream=None):
+        _check(lib().svd_verify_distill(ctypes.byref(self.args), self.ws.ptr, self.ws.nbytes,
+                                        _stream(stream)), "svd_verify_distill")
+        return self
+
+    def outputs(self) -> dict:
+        out = dict(bhat=self.bhat, bk=self.bk, accept_len=self.accept_len, emitted=self.emitted,
+                   n_emitted=self.n_emitted, loss_rows=self.loss_rows, loss_total=self.loss_total,
+                   dlogits=self.dlogits)
+        if self.row_info is not None:
+            out["row_info"] = self.row_info
+        return out
+
+
+def svd_verify_distill(D, T, **kw) -> dict:
+    """a1-a5 in one call; keyword arguments as in :class:`VerifyDistill`."""
+    return VerifyDistill(D, T, **kw)().outputs()
+
+
+def svd_selftest_wait_timeout(ws: Workspace, limit_ns: int, stream=None) -> None:
+    _check(lib().svd_selftest_wait_timeout(ws.ptr, ws.nbytes, int(limit_ns), _stream(stream)),
+           "svd_selftest_wait_timeout")
+
+
+INF = math.inf

@@ -1,0 +1,119 @@
+// svd_internal.h -- kernel parameter blocks, workspace layout and launch entry points shared by
+// the C ABI layer (svd_api.cu) and the kernels (length_head.cu, verify_distill.cu).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/svd.h"
+
+namespace svd {
+
+// ------------------------------------------------------------------------------------------
+// Workspace layout (all sections 256-byte aligned).  Everything except the status word is
+// returned to zero by the kernel that used it.
+// ------------------------------------------------------------------------------------------
+struct WsHeader {
+    uint32_t status;       // first device-side error (svd_status), sticky until read
+    uint32_t head_ticket;  // length head: CTAs finished
+    uint32_t loss_ticket;  // row pass: sequences finished
+    uint32_t pad[61];
+};
+static_assert(sizeof(WsHeader) == 256, "header is one 256-byte line");
+
+constexpr int kHeadTileM = 64;   // hidden units per length-head CTA
+constexpr int kHeadTileB = 16;   // sequences per length-head CTA
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+    size_t seq_ticket, rec, seq_loss, zpart, total;
+};
+
+__host__ __device__ inline WsLayout ws_layout(int B, int k, int kt, int M) {
+    (void)k;
+    WsLayout L;
+    size_t off = sizeof(WsHeader);
+    L.seq_ticket = off;
+    off = align256(off + sizeof(uint32_t) * (size_t)B);
+    L.rec = off;
+    off = align256(off + sizeof(svd_row_info) * (size_t)B * (size_t)kt);
+    L.seq_loss = off;
+    off = align256(off + sizeof(float) * (size_t)B);
+    L.zpart = off;
+    const int mt = M > 0 ? (M + kHeadTileM - 1) / kHeadTileM : 0;
+    off = align256(off + sizeof(float) * (size_t)mt * (size_t)B);
+    L.total = off;
+    return L;
+}
+
+// ------------------------------------------------------------------------------------------
+// length head
+// ------------------------------------------------------------------------------------------
+struct HeadParams {
+    const uint16_t* h;
+    const uint16_t* W1;
+    const float* b1;
+    const uint16_t* w2;
+    float b2;
+    int B, H, M, k;
+    float gamma;
+    int rnd;
+    float* bhat;
+    int32_t* bk;
+    WsHeader* hdr;
+    float* zpart;  // [ceil(M/64), B]
+};
+
+// ------------------------------------------------------------------------------------------
+// row pass (verify + distill)
+// ------------------------------------------------------------------------------------------
+enum : int {
+    kFlagVerify = 1,
+    kFlagDistill = 2,
+    kFlagStochastic = 4,
+};
+
+struct RowParams {
+    const uint16_t* D;
+    const uint16_t* T;
+    const int32_t* draft;
+    const int32_t* bk;
+    int B, k, kt, V;
+    int chunk;         // logit elements per CTA of a row cluster (multiple of 8)
+    int flags;
+    int aligned;       // 1: TMA bulk staging and vector stores; 0: plain loads / stores
+    float tau, inv_tau, k2;  // k2 = log2(e) / tau
+    uint64_t seed, step;
+    float lambda, clip_c, grad_scale;
+    int dl_fp32;
+    void* dlogits;
+    float* loss_rows;
+    float* loss_total;
+    int32_t* accept_len;
+    int32_t* emitted;
+    int32_t* n_emitted;
+    svd_row_info* row_info;
+    WsHeader* hdr;
+    uint32_t* seq_ticket;
+    svd_row_info* rec;
+    float* seq_loss;
+    uint64_t wait_limit_ns;
+};
+
+// Launchers (return cudaError_t as int; 0 = success).
+int launch_length_head(const HeadParams& p, void* stream);
+int launch_row_pass(const RowParams& p, void* stream);
+int launch_wait_timeout_selftest(WsHeader* hdr, uint64_t limit_ns, void* stream);
+
+// Cluster geometry chosen for a vocabulary size.
+struct RowGeometry {
+    int variant;   // 0: 128 threads x 2 vectors; 1: 512 threads x 5 vectors
+    int threads;
+    int cluster;   // CTAs per row
+    int chunk;     // elements per CTA
+    size_t smem;   // dynamic shared memory per CTA
+};
+bool row_geometry(int V, RowGeometry* g);
+
+}  // namespace svd
