@@ -224,6 +224,8 @@ def main():
     ap.add_argument("--cpu-seqs", type=int, default=0, help="oracle sample size (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(syn.WORKLOADS),
+                    help="profiling only: the reported bench line is the default workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -240,20 +242,28 @@ def main():
         raise SystemExit("bench.py needs a CUDA device (the CUDA path has no CPU fallback)")
     torch.cuda.set_device(info.local_rank)
     dev = torch.device("cuda", info.local_rank)
-    w = syn.WORKLOADS[WORKLOAD]
+    w = syn.WORKLOADS[args.workload]
     wr, host, d = build_inputs(w, parallel.rank_seed(0, info.rank) if info.rank else 0, dev)
     stream = torch.cuda.current_stream(dev)
 
     ws = api.Workspace(w.B, w.k, w.kt, w.M, device=dev)
+    draft = None
+    if w.mode == 1:
+        draft = syn.sample_draft_tokens(host["D"], w.tau, 77).to(dev)
+    head = (d["h"], d["W1"], d["b1"], d["w2"], d["b2"])
+    # the product call: length head + row pass in one svd_verify_distill (programmatic launch)
+    fused = api.VerifyDistill(d["D"], d["T"], head=head, draft_tok=draft, mode=w.mode,
+                              temperature=w.tau, seed=w.philox_seed, lam=w.lam, clip_c=w.clip_c,
+                              ws=ws)
+    # the same two kernels launched separately, for per-kernel times (roofline of the row pass)
     bhat = torch.empty(w.B, dtype=torch.float32, device=dev)
-    bk = torch.empty(w.B, dtype=torch.int32, device=dev)
-    # the row pass reads b_k from the head's output buffer in place
-    vd = api.VerifyDistill(d["D"], d["T"], bk_in=bk, mode=w.mode, temperature=w.tau,
-                           seed=w.philox_seed, lam=w.lam, clip_c=w.clip_c, ws=ws)
-    vd.args.bk = api._ptr(bk)
-    vd.bk = bk
+    bk = fused.bk
+    rows_only = api.VerifyDistill(d["D"], d["T"], bk_in=bk, draft_tok=draft, mode=w.mode,
+                                  temperature=w.tau, seed=w.philox_seed, lam=w.lam,
+                                  clip_c=w.clip_c, ws=ws)
+    rows_only.args.bk = api._ptr(bk)   # read b_k in place: no copy
 
-    def step_head_into():
+    def head_only():
         api.lib().svd_length_head(api._ptr(d["h"]), api._ptr(d["W1"]), api._ptr(d["b1"]),
                                   api._ptr(d["w2"]), float(d["b2"]), w.B, w.H, w.M, w.k, 1.0,
                                   api.BK_CEIL, api._ptr(bhat), api._ptr(bk), ws.ptr, ws.nbytes,
@@ -261,18 +271,20 @@ def main():
 
     # ---------------------------------------------------------------- warm-up
     for _ in range(args.warmup):
-        step_head_into()
-        vd()
+        fused()
+        head_only()
+        rows_only()
     torch.cuda.synchronize()
     if api.svd_get_device_error(ws) != 0:
         raise SystemExit("device error during warm-up")
+    fused()
+    torch.cuda.synchronize()
     bk_host = bk.cpu().numpy()
-    acc_host = vd.accept_len.cpu().numpy()
-    ne_host = vd.n_emitted.cpu().numpy()
+    acc_host = fused.accept_len.cpu().numpy()
+    ne_host = fused.n_emitted.cpu().numpy()
 
     # ---------------------------------------------------------------- timed region (device)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     clocks = None if args.no_clocks else ClockSampler(dev.index if dev.index is not None else 0)
     if info.world > 1:
         torch.distributed.barrier()
@@ -283,23 +295,30 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for s in range(K):
-        ev[s][0].record(stream)
-        step_head_into()
-        ev[s][1].record(stream)
-        vd()
-        ev[s][2].record(stream)
+        fused()
     t_end.record(stream)
+    torch.cuda.synchronize()
+    # per-kernel durations: the same step as two separately timed launches
+    KB = min(K, 200)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(KB)]
+    for s in range(KB):
+        ev[s][0].record(stream)
+        head_only()
+        ev[s][1].record(stream)
+        rows_only()
+        ev[s][2].record(stream)
     torch.cuda.synchronize()
     clock_rec = clocks.stop() if clocks else None
     if info.world > 1:
         torch.distributed.barrier()
     total_ms = t_start.elapsed_time(t_end)
-    head_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
-    rows_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
+    head_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(KB)]
+    rows_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(KB)]
     ms_per_step = total_ms / K
     err = api.svd_get_device_error(ws)
     if err != 0:
         raise SystemExit("device error in the timed region: %s" % api.STATUS_NAMES.get(err))
+    vd = fused
 
     verified = float(bk_host.sum())
     accepted = float(acc_host.sum())
@@ -334,7 +353,6 @@ def main():
             d["D"].copy_(host["D"], non_blocking=True)
             d["T"].copy_(host["T"], non_blocking=True)
             d["h"].copy_(host["h"], non_blocking=True)
-            step_head_into()
             vd()
             for n, t in (("accept_len", vd.accept_len), ("emitted", vd.emitted),
                          ("n_emitted", vd.n_emitted), ("loss_total", vd.loss_total), ("bk", bk)):
@@ -362,7 +380,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
             "steps": K, "warmup": args.warmup, "ms_per_step": red["ms"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": w.B, "k": w.k, "kt": w.kt, "V": w.V, "H": w.H,
+            "config": {"workload": args.workload, "B": w.B, "k": w.k, "kt": w.kt, "V": w.V, "H": w.H,
                        "M": w.M, "mode": "greedy", "lambda": w.lam, "clip_c": w.clip_c,
                        "storage": "bf16 logits / bf16 gradient, fp32 arithmetic",
                        "l2": "inputs larger than L2 (%.2f GB of logits per step, no flush)"

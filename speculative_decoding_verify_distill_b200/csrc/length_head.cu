@@ -6,13 +6,13 @@
 // representation is mapped to a single scalar and converted linearly to the verification length,
 // gamma = 1.0; Referee Report minor comment 2: b_k = clamp(floor(bhat * k), 1, k)).
 //
-// The projection h [B,H] x W1^T [H,M] is a small dense contraction (2*B*H*M flops, e.g. 0.27
-// GFLOP at B=128, H=4096, M=256), run on the tensor cores with bf16 operands and fp32
-// accumulation.  Grid: one CTA per (16 sequences, 64 hidden units); the 8 warps of a CTA split
-// the H axis and their 16x64 partial tiles are summed in shared memory in a fixed order.  Each
-// CTA then applies bias, ReLU and its slice of w2, leaving one partial logit per sequence; the
-// last CTA to finish (atomic ticket, no waiting) adds the partials in tile order, applies the
-// sigmoid and the b_k map.
+// The projection h [B,H] x W1^T [H,M] is a small dense contraction (2*B*H*M flops, 0.27 GFLOP
+// at B=128, H=4096, M=256) on the tensor cores: bf16 operands, fp32 accumulation.  The grid is
+// (16-sequence tiles) x (64-unit tiles) x (K splits); each CTA stages its operand slices in
+// shared memory with 16-byte loads and its 8 warps each accumulate one 16x8 output tile.  Split
+// partials land in the workspace; the last CTA of an output tile (atomic ticket, no waiting) adds
+// them in split order, applies bias, ReLU and w2, and the last tile adds the per-tile logits in
+// tile order and applies the sigmoid and the b_k map.  Every sum has a fixed order.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -24,6 +24,9 @@ namespace svd {
 namespace {
 
 constexpr int kWarps = 8;
+constexpr int kKC = 256;          // K chunk staged in shared memory
+constexpr int kPad = 8;           // row padding (16 bytes): conflict-free fragment reads
+constexpr int kLd = kKC + kPad;
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
                                                const uint32_t (&b)[2]) {
@@ -34,108 +37,136 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Two consecutive bf16 elements (row r, columns c, c+1) of a [rows, cols] matrix; zero outside.
-__device__ __forceinline__ uint32_t load_pair(const uint16_t* m, int rows, int cols, int r, int c,
-                                              bool vec_ok) {
-    if (r >= rows) return 0u;
-    const uint16_t* src = m + static_cast<size_t>(r) * cols + c;
-    if (vec_ok && c + 1 < cols) return __ldg(reinterpret_cast<const uint32_t*>(src));
-    const uint32_t lo = c < cols ? __ldg(src) : 0u;
-    const uint32_t hi = c + 1 < cols ? __ldg(src + 1) : 0u;
-    return lo | (hi << 16);
+// rows x kKC tile of a [nrows, ncols] bf16 matrix into padded shared memory; zero outside
+// [0, nrows) x [c0, c1).
+__device__ __forceinline__ void stage_tile(uint16_t* dst, const uint16_t* src, int rows, int r0,
+                                           int nrows, int ncols, int c0, int c1, bool vec_ok) {
+    const int vecs = rows * (kKC / 8);
+    for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
+        const int r = v / (kKC / 8), cv = (v % (kKC / 8)) * 8;
+        const int gr = r0 + r, gc = c0 + cv;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (gr < nrows) {
+            const uint16_t* s = src + static_cast<size_t>(gr) * ncols + gc;
+            if (vec_ok && gc + 8 <= c1) {
+                val = __ldg(reinterpret_cast<const uint4*>(s));
+            } else {
+                uint16_t e[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) e[q] = (gc + q < c1) ? __ldg(s + q) : uint16_t(0);
+                val = make_uint4(e[0] | (uint32_t(e[1]) << 16), e[2] | (uint32_t(e[3]) << 16),
+                                 e[4] | (uint32_t(e[5]) << 16), e[6] | (uint32_t(e[7]) << 16));
+            }
+        }
+        *reinterpret_cast<uint4*>(dst + r * kLd + cv) = val;
+    }
 }
 
 }  // namespace
 
 __global__ void __launch_bounds__(kWarps * 32) length_head_kernel(const HeadParams p) {
-    __shared__ float part[kWarps][kHeadTileB][kHeadTileM + 1];
-    __shared__ float zrow[kHeadTileB][kWarps];
-    __shared__ int is_last;
+    // let the dependent row pass start its prologue (it waits for this grid before reading b_k)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ __align__(16) uint16_t hs[kHeadTileB * kLd];
+    __shared__ __align__(16) uint16_t ws[kHeadTileM * kLd];
+    __shared__ float pre[kHeadTileB][kHeadTileM + 1];
+    __shared__ int flag;
 
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int b0 = blockIdx.x * kHeadTileB, m0 = blockIdx.y * kHeadTileM;
+    const int bt = blockIdx.x, mt = blockIdx.y, kz = blockIdx.z;
+    const int b0 = bt * kHeadTileB, m0 = mt * kHeadTileM;
     const int g = lane >> 2, tq = lane & 3;
-    // 32-bit fragment loads need even row lengths and 4-byte aligned bases
-    const bool vec_ok = (p.H % 2 == 0) && ((reinterpret_cast<uintptr_t>(p.h) & 3) == 0) &&
-                        ((reinterpret_cast<uintptr_t>(p.W1) & 3) == 0);
+    const int k_lo = min(p.H, kz * p.ks), k_hi = min(p.H, k_lo + p.ks);
+    const bool vec_ok = (p.H % 8 == 0) && ((reinterpret_cast<uintptr_t>(p.h) & 15) == 0) &&
+                        ((reinterpret_cast<uintptr_t>(p.W1) & 15) == 0);
 
-    float acc[8][4];
-#pragma unroll
-    for (int n = 0; n < 8; ++n)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
-
-    const int ksteps = (p.H + 15) / 16;
-    for (int s = warp; s < ksteps; s += kWarps) {
-        const int k0 = s * 16 + 2 * tq;
-        uint32_t a[4];
-        a[0] = load_pair(p.h, p.B, p.H, b0 + g, k0, vec_ok);
-        a[1] = load_pair(p.h, p.B, p.H, b0 + g + 8, k0, vec_ok);
-        a[2] = load_pair(p.h, p.B, p.H, b0 + g, k0 + 8, vec_ok);
-        a[3] = load_pair(p.h, p.B, p.H, b0 + g + 8, k0 + 8, vec_ok);
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-            const int m = m0 + n * 8 + g;
-            uint32_t bf[2];
-            bf[0] = load_pair(p.W1, p.M, p.H, m, k0, vec_ok);
-            bf[1] = load_pair(p.W1, p.M, p.H, m, k0 + 8, vec_ok);
-            mma_bf16_16816(acc[n], a, bf);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int c0 = k_lo; c0 < k_hi; c0 += kKC) {
+        const int c1 = min(k_hi, c0 + kKC);
+        stage_tile(hs, p.h, kHeadTileB, b0, p.B, p.H, c0, c1, vec_ok);
+        stage_tile(ws, p.W1, kHeadTileM, m0, p.M, p.H, c0, c1, vec_ok);
+        __syncthreads();
+        const uint16_t* wrow = ws + (warp * 8 + g) * kLd;
+#pragma unroll 4
+        for (int kk = 0; kk < kKC; kk += 16) {
+            if (c0 + kk >= c1) break;
+            uint32_t a[4], bf[2];
+            a[0] = *reinterpret_cast<const uint32_t*>(hs + g * kLd + kk + 2 * tq);
+            a[1] = *reinterpret_cast<const uint32_t*>(hs + (g + 8) * kLd + kk + 2 * tq);
+            a[2] = *reinterpret_cast<const uint32_t*>(hs + g * kLd + kk + 2 * tq + 8);
+            a[3] = *reinterpret_cast<const uint32_t*>(hs + (g + 8) * kLd + kk + 2 * tq + 8);
+            bf[0] = *reinterpret_cast<const uint32_t*>(wrow + kk + 2 * tq);
+            bf[1] = *reinterpret_cast<const uint32_t*>(wrow + kk + 2 * tq + 8);
+            mma_bf16_16816(acc, a, bf);
         }
+        __syncthreads();
     }
-    // accumulator layout: acc[n][0..1] = (row g, cols n*8 + 2tq + {0,1}); [2..3] = row g + 8
-#pragma unroll
-    for (int n = 0; n < 8; ++n) {
-        part[warp][g][n * 8 + 2 * tq] = acc[n][0];
-        part[warp][g][n * 8 + 2 * tq + 1] = acc[n][1];
-        part[warp][g + 8][n * 8 + 2 * tq] = acc[n][2];
-        part[warp][g + 8][n * 8 + 2 * tq + 1] = acc[n][3];
-    }
-    __syncthreads();
-
-    // each warp owns two sequences of the tile; lanes cover the 64 hidden units in pairs
-    for (int rb = warp * 2; rb < warp * 2 + 2; ++rb) {
-        float zsum = 0.f;
+    // accumulator layout: acc[0..1] = (row g, cols 2tq + {0,1}); acc[2..3] = row g + 8
+    {
+        float* part = p.part + static_cast<size_t>(kz) * p.B * p.M;
+        const int m = m0 + warp * 8 + 2 * tq;
+        const int rows[2] = {b0 + g, b0 + g + 8};
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-            const int col = lane + 32 * h2;
-            const int m = m0 + col;
-            float a = 0.f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) a += part[w][rb][col];
-            if (m < p.M) {
-                if (p.b1) a += __ldg(p.b1 + m);
-                const float hid = fmaxf(a, 0.f);
-                const float w2 = __uint_as_float(static_cast<uint32_t>(__ldg(p.w2 + m)) << 16);
-                zsum = fmaf(w2, hid, zsum);
+            const int b = rows[h2];
+            if (b < p.B) {
+                if (m < p.M) part[static_cast<size_t>(b) * p.M + m] = acc[2 * h2];
+                if (m + 1 < p.M) part[static_cast<size_t>(b) * p.M + m + 1] = acc[2 * h2 + 1];
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) zsum += __shfl_xor_sync(0xffffffffu, zsum, o);
-        if (lane == 0) zrow[rb][0] = zsum;
+    }
+    // last split of this output tile reduces the partials in split order
+    __threadfence();
+    __syncthreads();
+    if (t == 0) {
+        const uint32_t old = atomicAdd(&p.tile_ticket[bt * gridDim.y + mt], 1u);
+        flag = (old + 1u == gridDim.z) ? 1 : 0;
     }
     __syncthreads();
-    if (t < kHeadTileB && b0 + t < p.B) p.zpart[static_cast<size_t>(blockIdx.y) * p.B + b0 + t] = zrow[t][0];
-
-    // last CTA to finish combines the partial logits of every tile
+    if (!flag) return;
+    __threadfence();
+    for (int o = t; o < kHeadTileB * kHeadTileM; o += blockDim.x) {
+        const int r = o / kHeadTileM, col = o % kHeadTileM;
+        const int b = b0 + r, m = m0 + col;
+        float a = 0.f;
+        if (b < p.B && m < p.M) {
+            for (int z = 0; z < static_cast<int>(gridDim.z); ++z)
+                a += __ldcg(p.part + (static_cast<size_t>(z) * p.B + b) * p.M + m);
+            if (p.b1) a += __ldg(p.b1 + m);
+            const float w2 = __uint_as_float(static_cast<uint32_t>(__ldg(p.w2 + m)) << 16);
+            a = w2 * fmaxf(a, 0.f);
+        }
+        pre[r][col] = a;
+    }
+    __syncthreads();
+    // per-sequence sum over this tile's 64 units (warp w: rows 2w, 2w+1; fixed shuffle order)
+    for (int r = warp * 2; r < warp * 2 + 2; ++r) {
+        float z = pre[r][lane] + pre[r][lane + 32];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        if (lane == 0 && b0 + r < p.B) p.zpart[static_cast<size_t>(mt) * p.B + b0 + r] = z;
+    }
+    if (t == 0) p.tile_ticket[bt * gridDim.y + mt] = 0u;
+    // last output tile combines the per-tile logits of every sequence
     __threadfence();
     __syncthreads();
     if (t == 0) {
         const uint32_t total = gridDim.x * gridDim.y;
         const uint32_t old = atomicAdd(&p.hdr->head_ticket, 1u);
-        is_last = (old + 1u == total) ? 1 : 0;
+        flag = (old + 1u == total) ? 2 : 0;
     }
     __syncthreads();
-    if (!is_last) return;
+    if (flag != 2) return;
     __threadfence();
     const int mtiles = gridDim.y;
     for (int b = t; b < p.B; b += blockDim.x) {
         float z = p.b2;
-        for (int mt = 0; mt < mtiles; ++mt) z += __ldcg(p.zpart + static_cast<size_t>(mt) * p.B + b);
+        for (int q = 0; q < mtiles; ++q) z += __ldcg(p.zpart + static_cast<size_t>(q) * p.B + b);
         const float bhat = 1.f / (1.f + expf(-z));
         const float target = p.gamma * bhat * static_cast<float>(p.k);
-        float r = p.rnd == 0 ? ceilf(target) : floorf(target);
+        const float r = p.rnd == 0 ? ceilf(target) : floorf(target);
         int bk = static_cast<int>(fminf(fmaxf(r, 1.f), static_cast<float>(p.k)));
-        if (!(r == r)) bk = 1;  // NaN guard (non-finite hidden states)
+        if (!(r == r)) bk = 1;  // non-finite hidden states
         if (p.bhat) p.bhat[b] = bhat;
         p.bk[b] = bk;
     }
@@ -143,7 +174,7 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_kernel(const HeadPara
 }
 
 int launch_length_head(const HeadParams& p, void* stream) {
-    dim3 grid((p.B + kHeadTileB - 1) / kHeadTileB, (p.M + kHeadTileM - 1) / kHeadTileM, 1);
+    dim3 grid((p.B + kHeadTileB - 1) / kHeadTileB, (p.M + kHeadTileM - 1) / kHeadTileM, p.nsplit);
     length_head_kernel<<<grid, kWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return static_cast<int>(cudaGetLastError());
 }

@@ -37,6 +37,8 @@ struct WsPtrs {
     svd_row_info* rec;
     float* seq_loss;
     float* zpart;
+    float* part;
+    uint32_t* tile_ticket;
 };
 
 WsPtrs carve(void* ws, int B, int k, int kt, int M) {
@@ -48,6 +50,8 @@ WsPtrs carve(void* ws, int B, int k, int kt, int M) {
     w.rec = reinterpret_cast<svd_row_info*>(base + L.rec);
     w.seq_loss = reinterpret_cast<float*>(base + L.seq_loss);
     w.zpart = reinterpret_cast<float*>(base + L.zpart);
+    w.part = reinterpret_cast<float*>(base + L.part);
+    w.tile_ticket = reinterpret_cast<uint32_t*>(base + L.tile_ticket);
     return w;
 }
 
@@ -64,7 +68,10 @@ svd_status run_head(const uint16_t* h, const uint16_t* W1, const float* b1, cons
     p.B = B; p.H = H; p.M = M; p.k = k;
     p.gamma = gamma; p.rnd = static_cast<int>(rnd);
     p.bhat = bhat_out; p.bk = bk_out;
-    p.hdr = w.hdr; p.zpart = w.zpart;
+    p.hdr = w.hdr; p.zpart = w.zpart; p.part = w.part; p.tile_ticket = w.tile_ticket;
+    p.nsplit = head_nsplit(B, M);
+    const int per = (H + p.nsplit - 1) / p.nsplit;
+    p.ks = (per + 15) & ~15;
     return from_cuda(launch_length_head(p, stream));
 }
 
@@ -73,7 +80,7 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
                     uint64_t step, float lambda, float clip_c, float grad_scale, int dl_fp32,
                     void* dlogits, float* loss_rows, float* loss_total, int32_t* accept_len,
                     int32_t* emitted, int32_t* n_emitted, svd_row_info* row_info, const WsPtrs& w,
-                    void* stream) {
+                    void* stream, int pdl = 0) {
     RowParams p;
     std::memset(&p, 0, sizeof p);
     p.D = D; p.T = T; p.draft = draft; p.bk = bk;
@@ -92,6 +99,7 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
     p.row_info = row_info;
     p.hdr = w.hdr; p.seq_ticket = w.seq_ticket; p.rec = w.rec; p.seq_loss = w.seq_loss;
     p.wait_limit_ns = kWaitLimitNs;
+    p.pdl = pdl;
     return from_cuda(launch_row_pass(p, stream));
 }
 
@@ -209,7 +217,7 @@ svd_status svd_verify_distill(const svd_verify_distill_args* a, void* ws, size_t
     return run_rows(a->D, a->T, a->draft_tok, bk, a->B, a->k, a->kt, a->V, flags, a->temperature,
                     a->seed, a->step, a->lambda, a->clip_c, a->grad_scale, a->dlogits_fp32,
                     a->dlogits, a->loss_rows, a->loss_total, a->accept_len, a->emitted,
-                    a->n_emitted, a->row_info, w, stream);
+                    a->n_emitted, a->row_info, w, stream, head ? 1 : 0);
 }
 
 svd_status svd_get_device_error(void* ws, void* stream) {

@@ -26,8 +26,16 @@ constexpr int kHeadTileB = 16;   // sequences per length-head CTA
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// K splits of the length-head contraction: enough CTAs to cover the SMs twice over.
+__host__ __device__ inline int head_nsplit(int B, int M) {
+    if (B <= 0 || M <= 0) return 0;
+    const int tiles = ((B + kHeadTileB - 1) / kHeadTileB) * ((M + kHeadTileM - 1) / kHeadTileM);
+    int n = (296 + tiles - 1) / tiles;
+    return n < 1 ? 1 : (n > 16 ? 16 : n);
+}
+
 struct WsLayout {
-    size_t seq_ticket, rec, seq_loss, zpart, total;
+    size_t seq_ticket, rec, seq_loss, zpart, part, tile_ticket, total;
 };
 
 __host__ __device__ inline WsLayout ws_layout(int B, int k, int kt, int M) {
@@ -40,9 +48,14 @@ __host__ __device__ inline WsLayout ws_layout(int B, int k, int kt, int M) {
     off = align256(off + sizeof(svd_row_info) * (size_t)B * (size_t)kt);
     L.seq_loss = off;
     off = align256(off + sizeof(float) * (size_t)B);
-    L.zpart = off;
     const int mt = M > 0 ? (M + kHeadTileM - 1) / kHeadTileM : 0;
+    const int bt = (B + kHeadTileB - 1) / kHeadTileB;
+    L.zpart = off;
     off = align256(off + sizeof(float) * (size_t)mt * (size_t)B);
+    L.part = off;
+    off = align256(off + sizeof(float) * (size_t)head_nsplit(B, M) * (size_t)B * (size_t)(M > 0 ? M : 0));
+    L.tile_ticket = off;
+    off = align256(off + sizeof(uint32_t) * (size_t)bt * (size_t)mt);
     L.total = off;
     return L;
 }
@@ -62,7 +75,10 @@ struct HeadParams {
     float* bhat;
     int32_t* bk;
     WsHeader* hdr;
-    float* zpart;  // [ceil(M/64), B]
+    float* zpart;            // [ceil(M/64), B] per-tile logits
+    float* part;             // [nsplit, B, M] split partials of W1 h
+    uint32_t* tile_ticket;   // [ceil(B/16) * ceil(M/64)]
+    int nsplit, ks;          // K splits and columns per split
 };
 
 // ------------------------------------------------------------------------------------------
@@ -99,6 +115,7 @@ struct RowParams {
     svd_row_info* rec;
     float* seq_loss;
     uint64_t wait_limit_ns;
+    int pdl;           // launched as a programmatic dependent of the length head
 };
 
 // Launchers (return cudaError_t as int; 0 = success).

@@ -1,7 +1,7 @@
 // verify_distill.cu -- the fused row pass: truncated verification (greedy / stochastic) and the
 // clipped reverse-KL + CE distillation loss with its gradient, one HBM read per logit row.
 //
-// What it computes (AdaFlash, Pith review page "What carries the argument", Axiom & Free-
+// What it computes (AdaFlash; Pith review page "What carries the argument", Axiom & Free-
 // Parameter Ledger, Referee Report major comment 2; Pith verdict record load_bearing_attack):
 // for every sequence b the first b_k draft rows are verified against the target rows, the
 // acceptance length a_b and the emitted tokens follow the standard speculative-decoding rule,
@@ -9,23 +9,25 @@
 // zero gradient row.
 //
 // Design (B200, sm_100a):
-//   * Persistent grid of thread-block clusters; one cluster owns one logit row at a time, each
-//     CTA of the cluster a contiguous slice ("chunk") of the vocabulary.  Work items are the
-//     verified rows (position-major), the bonus rows, then the rows that are only zero-filled;
-//     cluster c takes items c, c + #clusters, ...
-//   * A slice of D and T is staged into shared memory by 1-D bulk copies (cp.async.bulk, no
-//     multicast) completing on mbarriers; the next item's copies are issued as soon as the
-//     current slice has been consumed, so HBM reads stream while the cluster finishes the row.
-//   * Pass A (from the staging buffer): per-thread online max / sum of exp for D and T, exp
-//     values e_v of D kept in registers, delta_v = D_v - T_v kept in shared memory (fp32).
-//     Cluster reduction #1 over distributed shared memory gives lse(D/tau), lse(T/tau).
-//   * Pass B (registers + shared memory): sum of d_v = q_v s_v, the rare clipped entries, and in
-//     stochastic mode the residual masses as 2^-48 fixed-point integers (exact, order-free
-//     prefix sums).  Argmax (lowest id) is resolved lazily by the threads that hold the row max.
-//     Cluster reduction #2.
+//   * Persistent grid of thread-block clusters; a cluster owns one logit row at a time, each of
+//     its CTAs a contiguous slice ("chunk") of the vocabulary, and each warp of a CTA a
+//     contiguous run of 16-byte vectors of that slice.  Work items are the verified rows
+//     (position-major), the bonus rows, then the rows that are only zero-filled; cluster c takes
+//     items c, c + #clusters, ...  Every warp decodes the item sequence itself (b_k is cached in
+//     shared memory), so warps never wait on each other inside a CTA.
+//   * Each warp stages its run of D and T with its own 1-D bulk copies (cp.async.bulk, no
+//     multicast) completing on its own mbarrier, and refills the same buffer with the next item
+//     as soon as it has read it: HBM reads stream while the cluster finishes the row.
+//   * Pass A: per-thread online max / sum of exp of D and T; exp values of D stay in registers,
+//     delta = D - T goes to shared memory (fp32).  Per-warp partials, cluster barrier #1, then
+//     every warp reads all partials of the cluster over DSMEM and has lse(D/tau), lse(T/tau).
+//   * Pass B: sum of d_v = q_v s_v, the rare clipped entries, and in stochastic mode the sample
+//     masses as 2^-48 fixed-point integers (exact, associative prefix sums).  Argmax (lowest id)
+//     is resolved lazily by the threads that hold the row maximum.  Cluster barrier #2.
 //   * Pass C: dL/dD = q (P + Q delta) (+ clipped and hard-label corrections), 16-byte stores.
-//   * The CTA that completes the last row of a sequence (atomic ticket; nothing ever waits on
-//     another CTA) runs the warp-ballot acceptance scan and writes the sequence's outputs.
+//   * Rank 0 of the cluster completes the row record one row later (off the critical path); the
+//     CTA that records the last row of a sequence (atomic ticket, nothing waits on another CTA)
+//     runs the warp-ballot acceptance scan and writes the sequence's outputs.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -38,55 +40,57 @@ namespace svd {
 namespace {
 
 constexpr uint32_t kNone = 0xffffffffu;
-#define kNegInf (-__int_as_float(0x7f800000))  // -inf
+#define kNegInf (-__int_as_float(0x7f800000))
+#define kQNaN (__int_as_float(0x7fc00000))
 
 enum ItemKind : int { kItemNone = 0, kItemRow = 1, kItemBonus = 2, kItemZero = 3 };
 
-// Per-CTA exchange slot, read and written across the cluster through DSMEM.
-struct alignas(16) Slot {
-    float mD, sD, mT, sT;                   // reduction #1: max / sum-exp (relative to max)
-    float sum_d, clip_d, clip_q, n_clip;    // reduction #2: reverse-KL partials
-    unsigned long long mass;                // reduction #2: this CTA's sample mass (2^-48 units)
-    unsigned long long mass2;               // fallback reduction: mass of p (2^-48 units)
-    uint32_t argD, argT;                    // rank 0: lowest index holding the row max
-    uint32_t tok;                           // rank 0: sampled token
-    float ce;                               // rank 0: -log q_y from the owner of y
+// Per-warp / per-CTA partials of the two cluster reductions.  Sums are relative to the maxima
+// they travel with (exp(x - m) in the log2-scaled domain).
+struct alignas(16) Part1 {
+    float mD, sD, sDd, dmax;   // max D, sum exp, sum exp * (D - T), max (D - T)
+    float mT, sT, pad0, pad1;  // max T, sum exp
 };
-
-// Values every thread of the CTA needs for the current row.
-struct RowG {
-    float MD, MT;        // row maxima of D and T (bf16 values)
-    float lseD, lseT;    // log sum exp(x / tau)
-    float L2D, L2T;      // lse * log2(e)
-    float dl;            // lseD - lseT
-    float P, Q, Pc, hardc;  // gradient coefficients
-    float ratio, u0, u1;
-    int acc;             // stochastic decision (or greedy decision once known)
-    int do_sample;       // stochastic: this row draws a token
-    int attempt_p;       // residual mass was zero: sample from p instead
-    uint32_t x, y;
-    float Dx, Tx;
-    unsigned long long R, off;  // total mass of the row, mass before this CTA's slice
-    unsigned long long tgt;     // sample point in [0, R)
-    float sum_d, clip_d, n_clip;
+struct alignas(16) Part2 {
+    float clip_d, clip_q, n_clip, pad0;    // clipped reverse-KL entries
+    unsigned long long mass;               // sample mass (2^-48 units)
+    unsigned long long pad1;
+};
+// Deposit targets in rank 0, double-buffered by row parity (read one row later).
+struct alignas(16) Deposit {
+    uint32_t argD, argT;       // lowest index holding the row max (red.min)
+    uint32_t tok;              // sampled token (red.min)
+    float ce;                  // -log q_y, from the owner of y
+};
+// Row values rank 0 keeps until the record is completed.
+struct Pending {
+    int b, i, kind;
+    int x, y, acc, do_sample;
+    float ratio, lseD, lseT, kc;
 };
 
 template <int NW>
 struct Ctl {
-    Slot slot;
-    RowG g;
-    float wred[NW][4];
-    unsigned long long wmass[NW];
-    int hist[34];
-    int cumV[34], cumZ[34];
-    int totV, totB, totZ;
-    int kind, b, i;          // current item
-    int nkind, nb, ni;       // next item
-    int fin;                 // this CTA completed a sequence
+    Part1 p1[NW];              // per-warp partials (local)
+    Part2 p2[NW];
+    Part1 cta1;                // CTA partials, read by every warp of the cluster over DSMEM
+    Part2 cta2;
+    Part2 cta3;                // fallback reduction (residual mass zero: sample from p)
+    unsigned long long wpre[NW];  // exclusive prefix of the warps' sample masses in this CTA
+    Deposit dep[2];
+    Pending pend;
+    int wscan[NW];             // prologue scan of the loaded-row counts
 };
 
-__device__ __forceinline__ int get_bk(const RowParams& p, int b) {
-    int n = __ldg(p.bk + b);
+// Batches up to this size keep b_k and the prefix of loaded rows per sequence in shared memory
+// (compact item list); larger batches walk the uncompacted (sequence, row) slots.
+constexpr int kCompactMaxB = 4096;
+
+struct Item {
+    int kind, b, i;
+};
+
+__device__ __forceinline__ int clamp_bk(const RowParams& p, int n) {
     if (n < 1 || n > p.k) {
         set_device_error(&p.hdr->status, SVD_ERR_INVALID_ARG);
         n = n < 1 ? 1 : p.k;
@@ -94,57 +98,54 @@ __device__ __forceinline__ int get_bk(const RowParams& p, int b) {
     return n;
 }
 
-__device__ __forceinline__ bool zero_row_pred(const RowParams& p, int n, int i, bool verify) {
-    // dlogits rows that only need zeros: i >= b_k, except the bonus row b_k (zeroed by its item)
-    return i < p.k && (verify ? (n < i) : (n <= i));
+// Loaded rows of a sequence: its verified rows, plus the bonus row when b_k < kt.
+__device__ __forceinline__ int loaded_rows(int n, int kt, bool verify) {
+    return n + ((verify && n < kt) ? 1 : 0);
 }
 
-// Lane that holds the r-th (0-based) sequence satisfying pred, found by warp ballots.
-template <typename Pred>
-__device__ int warp_select_rth(int B, int r, Pred pred) {
-    const int lane = threadIdx.x & 31;
-    for (int c = 0; c < B; c += 32) {
-        const int b = c + lane;
-        const bool q = b < B && pred(b);
-        const uint32_t m = __ballot_sync(0xffffffffu, q);
-        const int cnt = __popc(m);
-        if (r < cnt) {
-            const bool mine = q && __popc(m & ((1u << lane) - 1u)) == r;
-            const uint32_t who = __ballot_sync(0xffffffffu, mine);
-            return c + __ffs(who) - 1;
+// Gradient rows that only need zeros: i >= b_k, except the bonus row b_k (zeroed by its item).
+__device__ __forceinline__ bool zero_row_pred(int k, int n, int i, bool verify) {
+    return i < k && (verify ? (n < i) : (n <= i));
+}
+
+// b_k of sequence b: from shared memory (compact mode) or global memory (clamped).
+struct BkView {
+    const int* s;       // shared copy, or nullptr
+    const int32_t* g;   // global
+    __device__ __forceinline__ int operator()(const RowParams& p, int b) const {
+        return s ? s[b] : clamp_bk(p, __ldg(g + b));
+    }
+};
+
+// Loaded item w of the whole batch.  Compact mode: w indexes the list of loaded rows ordered by
+// sequence (prefix sums in shared memory, binary search).  Otherwise w is a (sequence, row) slot
+// and holes decode to kItemNone.
+__device__ __forceinline__ Item decode_loaded(const RowParams& p, const int* spre, const BkView& bkv,
+                                              int w, bool verify) {
+    Item it{kItemNone, -1, -1};
+    if (spre) {
+        if (w >= spre[p.B]) return it;
+        int lo = 0, hi = p.B;  // largest b with spre[b] <= w
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (spre[mid] <= w) lo = mid; else hi = mid;
         }
-        r -= cnt;
+        const int i = w - spre[lo];
+        const int n = bkv(p, lo);
+        it = Item{i < n ? kItemRow : kItemBonus, lo, i};
+    } else {
+        if (w >= p.B * p.kt) return it;
+        const int b = w / p.kt, i = w % p.kt;
+        const int n = bkv(p, b);
+        if (i < n) it = Item{kItemRow, b, i};
+        else if (verify && i == n) it = Item{kItemBonus, b, i};
     }
-    return -1;
+    return it;
 }
 
-// Decodes work item w into (kind, b, i); executed by a full warp.
-template <int NW>
-__device__ void decode_item(const RowParams& p, Ctl<NW>& c, int w, bool verify, int* kind, int* b,
-                            int* i) {
-    *kind = kItemNone; *b = -1; *i = -1;
-    if (w < c.totV) {
-        int pos = 0;
-        while (c.cumV[pos + 1] <= w) ++pos;
-        const int r = w - c.cumV[pos];
-        *b = warp_select_rth(p.B, r, [&](int s) { return get_bk(p, s) > pos; });
-        *i = pos;
-        *kind = kItemRow;
-    } else if (w < c.totV + c.totB) {
-        const int r = w - c.totV;
-        *b = warp_select_rth(p.B, r, [&](int s) { return get_bk(p, s) < p.kt; });
-        *i = get_bk(p, *b);
-        *kind = kItemBonus;
-    } else if (w < c.totV + c.totB + c.totZ) {
-        const int wz = w - c.totV - c.totB;
-        int pos = 0;
-        while (c.cumZ[pos + 1] <= wz) ++pos;
-        const int r = wz - c.cumZ[pos];
-        *b = warp_select_rth(p.B, r,
-                             [&](int s) { return zero_row_pred(p, get_bk(p, s), pos, verify); });
-        *i = pos;
-        *kind = kItemZero;
-    }
+// Number of loaded-item slots to walk (compact: exact count; otherwise all slots).
+__device__ __forceinline__ int loaded_slots(const RowParams& p, const int* spre) {
+    return spre ? spre[p.B] : p.B * p.kt;
 }
 
 // (max, sum) pairs of exp sums relative to their max, merged in the log2-scaled domain.
@@ -177,15 +178,79 @@ __device__ __forceinline__ unsigned long long scale_mass(unsigned long long R, u
     return (lo >> 24) | (hi << 40);
 }
 
+__device__ __forceinline__ void dsmem_ld4(uint32_t a, float (&v)[4]) {
+    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+                 : "r"(a)
+                 : "memory");
+}
+__device__ __forceinline__ unsigned long long dsmem_ld_u64(uint32_t a) {
+    unsigned long long v;
+    asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+// Scale factor that moves a sum relative to max m onto the common max M (0 for empty sums).
+__device__ __forceinline__ float rescale(float m, float M, float k2) {
+    return m == kNegInf ? 0.f : fast_exp2((m - M) * k2);
+}
+// Reduces per-lane Part1 values over the warp: maxima first, then one rescale per lane, then
+// plain sums; every lane ends with the result.
+__device__ __forceinline__ Part1 warp_reduce_part1(const Part1& a, float k2) {
+    Part1 r;
+    r.mD = warp_max(a.mD);
+    r.mT = warp_max(a.mT);
+    r.dmax = warp_max(a.dmax);
+    const float cD = rescale(a.mD, r.mD, k2), cT = rescale(a.mT, r.mT, k2);
+    r.sD = warp_sum(a.sD * cD);
+    r.sDd = warp_sum(a.sDd * cD);
+    r.sT = warp_sum(a.sT * cT);
+    r.pad0 = r.pad1 = 0.f;
+    return r;
+}
+__device__ __forceinline__ Part1 empty_part1() {
+    Part1 r;
+    r.mD = r.mT = r.dmax = kNegInf;
+    r.sD = r.sDd = r.sT = 0.f;
+    r.pad0 = r.pad1 = 0.f;
+    return r;
+}
+__device__ __forceinline__ float sum8(const float (&v)[8]) {
+    return ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+}
+__device__ __forceinline__ float max8f(const float (&v)[8]) {
+    return fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
+}
+
+__device__ __forceinline__ void warp_inclusive_scan_u64(unsigned long long& x) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+}
+
 }  // namespace
 
 template <int NT, int NV>
 __host__ __device__ constexpr size_t ctl_offset() {
+    // staging D, T: NV*NT uint4 each | delta planes: 2*NV*NT float4 | one barrier per warp
     return (static_cast<size_t>(NV) * NT * 16 * 2 + static_cast<size_t>(NV) * NT * 32 +
-            static_cast<size_t>(NV) * 8 + 127) & ~static_cast<size_t>(127);
+            static_cast<size_t>(NT / 32) * 8 + 127) & ~static_cast<size_t>(127);
 }
 
-template <int NT, int NV, bool DISTILL, bool STOCH>
+template <int NT, int NV, bool DISTILL, bool STOCH, bool ALIGNED>
 __global__ void __launch_bounds__(NT, 1) row_pass_kernel(const RowParams p) {
     constexpr int NW = NT / 32;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -194,672 +259,713 @@ __global__ void __launch_bounds__(NT, 1) row_pass_kernel(const RowParams p) {
     float4* dplane = reinterpret_cast<float4*>(stageT + NV * NT);
     uint64_t* full = reinterpret_cast<uint64_t*>(dplane + 2 * NV * NT);
     Ctl<NW>& c = *reinterpret_cast<Ctl<NW>*>(smem_raw + ctl_offset<NT, NV>());
+    // compact mode: b_k [B] and the prefix of loaded rows [B + 1] follow the control block
+    int* sbk = reinterpret_cast<int*>(smem_raw + ctl_offset<NT, NV>() + ((sizeof(Ctl<NW>) + 15) & ~size_t(15)));
+    int* spre = sbk + p.B;
 
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const uint32_t rank = cluster_rank();
-    const uint32_t CL = cluster_size();
+    const int CL = static_cast<int>(cluster_size());
     const int cid = static_cast<int>(cluster_id_x());
     const int ncl = static_cast<int>(num_clusters_x());
     const bool verify = (p.flags & kFlagVerify) != 0;
-    const bool need_lse = DISTILL || STOCH;
-    const int V = p.V;
+    constexpr bool need_lse = DISTILL || STOCH;
+    const int V = p.V, k = p.k, kt = p.kt;
     const int v0 = static_cast<int>(rank) * p.chunk;
     const int len = max(0, min(p.chunk, V - v0));
     const int nvec = (len + 7) >> 3;
+    // this warp's contiguous run of vectors: [wv0, wv0 + wcnt)
+    const int vpw = (nvec + NW - 1) / NW;
+    const int wv0 = min(nvec, warp * vpw);
+    const int wcnt = max(0, min(nvec, wv0 + vpw) - wv0);
     const float k2 = p.k2, itau = p.inv_tau;
+    uint4* myD = stageD + warp * NV * 32;
+    uint4* myT = stageT + warp * NV * 32;
 
     // ---------------------------------------------------------------- prologue
     if (t == 0) {
-        for (int j = 0; j < NV; ++j) mbar_init(&full[j], 1);
+        for (int q = 0; q < NW; ++q) mbar_init(&full[q], 1);
         fence_mbar_init();
-        c.slot.argD = kNone;
-        c.slot.argT = kNone;
-        c.slot.tok = kNone;
-        c.slot.ce = 0.f;
+        for (int q = 0; q < 2; ++q) {
+            c.dep[q].argD = kNone;
+            c.dep[q].argT = kNone;
+            c.dep[q].tok = kNone;
+            c.dep[q].ce = 0.f;
+        }
     }
-    if (t < 34) c.hist[t] = 0;
+    // Vectors past the end of a warp's run hold a finite sentinel (the most negative bf16) in
+    // both D and T: its exp is 0 and D - T is 0, so the passes below run straight-line code
+    // over all NV rounds with no per-vector branches.  The bulk copies never touch this tail.
+    {
+        const uint4 sent = make_uint4(0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu);
+        for (int lv = wcnt + lane; lv < NV * 32; lv += 32) {
+            myD[lv] = sent;
+            myT[lv] = sent;
+        }
+    }
     __syncthreads();
-    // histogram of b_k -> item counts
-    for (int b = t; b < p.B; b += NT) atomicAdd(&c.hist[get_bk(p, b)], 1);
-    __syncthreads();
-    if (t == 0) {
-        const int k = p.k;
-        c.cumV[0] = 0;
-        c.cumZ[0] = 0;
-        for (int i = 0; i < k; ++i) {
-            int cv = 0, cz = 0;
-            for (int n = 1; n <= k; ++n) {
-                if (n > i) cv += c.hist[n];
-                if (DISTILL && zero_row_pred(p, n, i, verify)) cz += c.hist[n];
+    // behind the length head (programmatic dependent launch) the prologue above overlapped its
+    // tail; b_k is read only after the head's writes are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const bool compact = p.B <= kCompactMaxB;
+    if (compact) {
+        // b_k and the exclusive prefix of loaded rows per sequence, in shared memory
+        int carry = 0;
+        for (int c0 = 0; c0 < p.B; c0 += NT) {
+            const int b = c0 + t;
+            int n = 0, L = 0;
+            if (b < p.B) {
+                n = clamp_bk(p, __ldg(p.bk + b));
+                L = loaded_rows(n, kt, verify);
+                sbk[b] = n;
             }
-            c.cumV[i + 1] = c.cumV[i] + cv;
-            c.cumZ[i + 1] = c.cumZ[i] + cz;
+            int incl = L;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane == 31) c.wscan[warp] = incl;
+            __syncthreads();
+            int before = 0, tot = 0;
+            for (int q = 0; q < NW; ++q) {
+                const int v = c.wscan[q];
+                if (q < warp) before += v;
+                tot += v;
+            }
+            if (b < p.B) spre[b] = carry + before + incl - L;
+            carry += tot;
+            __syncthreads();
         }
-        for (int i = k; i < 33; ++i) {
-            c.cumV[i + 1] = c.cumV[i] + 0x3fffffff;  // sentinel: never reached by a valid w
-            c.cumZ[i + 1] = c.cumZ[i] + 0x3fffffff;
-        }
-        c.totV = c.cumV[k];
-        c.totZ = c.cumZ[k];
-        c.totB = verify ? (p.B - (p.kt == k ? c.hist[k] : 0)) : 0;
+        if (t == 0) spre[p.B] = carry;
     }
     __syncthreads();
+    cluster_sync();  // barriers, deposit slots and the item list ready everywhere
 
-    uint32_t phase = 0;   // parity of the staging barriers for the next loaded item
-    bool wait_dead = false;  // a bounded wait ran out: skip later waits so the kernel finishes
+    const BkView bkv{compact ? sbk : nullptr, p.bk};
+    const int* list = compact ? spre : nullptr;
+    const int nslots = loaded_slots(p, list);
+    // the cluster's loaded items are slots cid, cid + ncl, ...; holes are skipped
+    auto next_loaded = [&](int& w) -> Item {
+        while (w < nslots) {
+            const Item it = decode_loaded(p, list, bkv, w, verify);
+            if (it.kind != kItemNone) return it;
+            w += ncl;
+        }
+        return Item{kItemNone, -1, -1};
+    };
 
-    auto issue_loads = [&](int kind, int b, int i) {
-        // thread 0 only; one phase of every staging barrier per loaded item
-        const uint16_t* Drow = p.D + (static_cast<size_t>(b) * p.k + i) * V + v0;
-        const uint16_t* Trow = p.T + (static_cast<size_t>(b) * p.kt + i) * V + v0;
-        for (int j = 0; j < NV; ++j) {
-            const int e0 = j * NT * 8;
-            const int n = max(0, min(len - e0, NT * 8));
-            const uint32_t bT = static_cast<uint32_t>(n) * 2u;         // target row: always
-            const uint32_t bD = (kind == kItemRow) ? bT : 0u;           // draft row: verified rows
-            mbar_arrive_expect_tx(&full[j], bD + bT);
-            if (bD) bulk_load(stageD + j * NT, Drow + e0, bD, &full[j]);
-            if (bT) bulk_load(stageT + j * NT, Trow + e0, bT, &full[j]);
+    // one warp's bulk copies of item `it` into its staging run (lane 0 only)
+    auto issue_loads = [&](const Item& it) {
+        const uint32_t bT = static_cast<uint32_t>(wcnt) * 16u;
+        const uint32_t bD = (it.kind == kItemRow) ? bT : 0u;
+        mbar_arrive_expect_tx(&full[warp], bD + bT);
+        if (bT) {
+            const size_t e0 = static_cast<size_t>(v0) + static_cast<size_t>(wv0) * 8;
+            if (bD) bulk_load(myD, p.D + (static_cast<size_t>(it.b) * k + it.i) * V + e0, bD, &full[warp]);
+            bulk_load(myT, p.T + (static_cast<size_t>(it.b) * kt + it.i) * V + e0, bT, &full[warp]);
         }
     };
 
     int w = cid;
-    if (warp == 0) {
-        int kind, b, i;
-        decode_item(p, c, w, verify, &kind, &b, &i);
-        if (lane == 0) { c.kind = kind; c.b = b; c.i = i; }
-    }
-    __syncthreads();
-    cluster_sync();  // barriers and slots initialised everywhere before any remote access
-    if (t == 0 && p.aligned && (c.kind == kItemRow || c.kind == kItemBonus))
-        issue_loads(c.kind, c.b, c.i);
+    Item cur = next_loaded(w);
+    if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
+    uint32_t phase = 0;          // parity of this warp's staging barrier
+    bool wait_dead = false;      // a bounded wait ran out: skip later waits so the kernel ends
+    int par = 0;                 // parity of the loaded rows (deposit double buffer)
+    bool pending = false;        // rank 0 owes the record of the previous loaded row
 
-    // ---------------------------------------------------------------- item loop
-    while (true) {
-        const int kind = c.kind, b = c.b, i = c.i;
-        if (kind == kItemNone) break;
-        const int wn = w + ncl;
-        if (warp == 0) {
-            int nk, nb, ni;
-            decode_item(p, c, wn, verify, &nk, &nb, &ni);
-            if (lane == 0) { c.nkind = nk; c.nb = nb; c.ni = ni; }
+    // rank 0, warp NW-1: complete the record of the previous loaded row (deposits now visible)
+    auto finish_record = [&]() {
+        const Pending& pd = c.pend;
+        const Deposit& dp = c.dep[par ^ 1];
+        int fin = 0;
+        if (lane == 0) {
+            const bool isRow = pd.kind == kItemRow;
+            svd_row_info r;
+            r.draft_token = pd.x;
+            r.target_argmax = pd.y;
+            r.accepted = pd.acc;
+            if (!verify) r.sample_token = -1;
+            else if (!STOCH) r.sample_token = pd.y;
+            else r.sample_token = (pd.do_sample && dp.tok != kNone) ? static_cast<int32_t>(dp.tok) : -1;
+            r.ratio = pd.ratio;
+            r.lse_draft = pd.lseD;
+            r.lse_target = pd.lseT;
+            float L = 0.f;
+            if (DISTILL && isRow) {
+                L = p.lambda * dp.ce + (1.f - p.lambda) * pd.kc;
+                if (p.loss_rows) p.loss_rows[static_cast<size_t>(pd.b) * k + pd.i] = L;
+            }
+            r.loss = L;
+            const size_t trow = static_cast<size_t>(pd.b) * kt + pd.i;
+            p.rec[trow] = r;
+            if (p.row_info) p.row_info[trow] = r;
+            Deposit& dw = c.dep[par ^ 1];
+            dw.argD = kNone;
+            dw.argT = kNone;
+            dw.tok = kNone;
+            dw.ce = 0.f;
+            __threadfence();
+            const int n = bkv(p, pd.b);
+            const uint32_t expected = static_cast<uint32_t>(loaded_rows(n, kt, verify));
+            const uint32_t old = atomicAdd(&p.seq_ticket[pd.b], 1u);
+            fin = (old + 1u == expected) ? 1 : 0;
         }
-        const size_t drow = static_cast<size_t>(b) * p.k + i;      // draft / gradient row
-        const size_t trow = static_cast<size_t>(b) * p.kt + i;     // target row
-
-        if (kind == kItemZero) {
-            // ---------------------------------------------------- zero-only gradient row
-            if (p.aligned) {
-                const uint4 z = make_uint4(0, 0, 0, 0);
-                if (p.dl_fp32) {
-                    float* g = static_cast<float*>(p.dlogits) + drow * V + v0;
-                    for (int e = t * 4; e < len; e += NT * 4) __stcs(reinterpret_cast<uint4*>(g + e), z);
-                } else {
-                    uint16_t* g = static_cast<uint16_t*>(p.dlogits) + drow * V + v0;
-                    for (int e = t * 8; e < len; e += NT * 8) __stcs(reinterpret_cast<uint4*>(g + e), z);
-                }
-            } else {
-                for (int e = t; e < len; e += NT) {
-                    if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + v0 + e] = 0.f;
-                    else static_cast<uint16_t*>(p.dlogits)[drow * V + v0 + e] = 0;
+        fin = __shfl_sync(0xffffffffu, fin, 0);
+        if (!fin) return;
+        // ---------------- sequence complete: acceptance scan, one lane per position
+        __threadfence();
+        const int b = pd.b;
+        const int n = bkv(p, b);
+        svd_row_info r;
+        r.draft_token = -1; r.target_argmax = -1; r.accepted = -1; r.sample_token = -1;
+        r.ratio = r.lse_draft = r.lse_target = kQNaN;
+        r.loss = 0.f;
+        auto is_processed = [&](int row) { return row < n || (verify && row == n && n < kt); };
+        if (lane < kt && is_processed(lane)) {
+            const svd_row_info* src = p.rec + static_cast<size_t>(b) * kt + lane;
+            r.draft_token = __ldcg(&src->draft_token);
+            r.target_argmax = __ldcg(&src->target_argmax);
+            r.accepted = __ldcg(&src->accepted);
+            r.sample_token = __ldcg(&src->sample_token);
+            r.loss = __ldcg(&src->loss);
+        } else if (lane < kt && p.row_info) {
+            p.row_info[static_cast<size_t>(b) * kt + lane] = r;  // unprocessed row
+        }
+        if (kt == 33 && lane == 0 && !is_processed(32) && p.row_info) {
+            svd_row_info u;
+            u.draft_token = u.target_argmax = u.accepted = u.sample_token = -1;
+            u.ratio = u.lse_draft = u.lse_target = kQNaN;
+            u.loss = 0.f;
+            p.row_info[static_cast<size_t>(b) * kt + 32] = u;
+        }
+        if (verify) {
+            const uint32_t accm = __ballot_sync(0xffffffffu, lane < n && r.accepted == 1);
+            int a = __ffs(~accm) - 1;
+            if (a > n || a < 0) a = n;
+            const int fix_row = a < n ? a : ((n < kt) ? n : -1);
+            int fix_tok = __shfl_sync(0xffffffffu, r.sample_token, fix_row < 0 ? 0 : (fix_row & 31));
+            if (fix_row >= 32)  // bonus row 32 (k = 32, kt = 33) has no lane of its own
+                fix_tok = __ldcg(&p.rec[static_cast<size_t>(b) * kt + 32].sample_token);
+            // lane q holds row q's record; slot k (= 32 at most) can only hold the fix token
+            if (lane < k + 1) {
+                int v = -1;
+                if (lane < a) v = r.draft_token;
+                else if (lane == a && fix_row >= 0) v = fix_tok;
+                p.emitted[static_cast<size_t>(b) * (k + 1) + lane] = v;
+            }
+            if (k == 32 && lane == 0)
+                p.emitted[static_cast<size_t>(b) * (k + 1) + 32] = (a == 32 && fix_row >= 0) ? fix_tok : -1;
+            if (lane == 0) {
+                p.accept_len[b] = a;
+                p.n_emitted[b] = a + (fix_row >= 0 ? 1 : 0);
+            }
+        }
+        if (DISTILL) {
+            if (p.loss_rows && lane >= n && lane < k) p.loss_rows[static_cast<size_t>(b) * k + lane] = 0.f;
+            float ls = 0.f;
+            for (int q = 0; q < n; ++q) ls += __shfl_sync(0xffffffffu, r.loss, q);
+            if (lane == 0) {
+                p.seq_loss[b] = ls;
+                p.seq_ticket[b] = 0u;
+                __threadfence();
+                const uint32_t old = atomicAdd(&p.hdr->loss_ticket, 1u);
+                if (old + 1u == static_cast<uint32_t>(p.B)) {
+                    __threadfence();
+                    float tot = 0.f;
+                    for (int s = 0; s < p.B; ++s) tot += __ldcg(p.seq_loss + s);
+                    *p.loss_total = tot;
+                    p.hdr->loss_ticket = 0u;
                 }
             }
-            __syncthreads();
-            if (t == 0) { c.kind = c.nkind; c.b = c.nb; c.i = c.ni; }
-            __syncthreads();
-            w = wn;
-            continue;
+        } else if (lane == 0) {
+            p.seq_ticket[b] = 0u;
         }
+    };
 
-        const bool isRow = (kind == kItemRow);
+    // ---------------------------------------------------------------- loaded rows
+    while (cur.kind != kItemNone) {
+        int wn = w + ncl;
+        const Item nxt = next_loaded(wn);
+        const int b = cur.b, i = cur.i;
+        const size_t drow = static_cast<size_t>(b) * k + i;      // draft / gradient row
+        const size_t trow = static_cast<size_t>(b) * kt + i;     // target row
+
+        const bool isRow = (cur.kind == kItemRow);
         const bool rowVerify = isRow && verify;
-        // draft token given by the caller: fetch D_x, T_x for the acceptance ratio
-        if (t == 0) {
-            uint32_t x = kNone;
-            float Dx = 0.f, Tx = 0.f;
-            if (rowVerify && p.draft != nullptr) {
-                const int xv = __ldg(p.draft + drow);
+        // caller's draft token and, in stochastic mode, D_x and T_x for the acceptance ratio
+        uint32_t x = kNone;
+        float Dx = 0.f, Tx = 0.f;
+        if (rowVerify && p.draft != nullptr) {
+            int xv = 0;
+            if (lane == 0) {
+                xv = __ldg(p.draft + drow);
                 if (xv < 0 || xv >= V) {
-                    set_device_error(&p.hdr->status, SVD_ERR_TOKEN_RANGE);
-                } else {
-                    x = static_cast<uint32_t>(xv);
-                    if (STOCH) {
-                        Dx = __uint_as_float(static_cast<uint32_t>(__ldg(p.D + drow * V + x)) << 16);
-                        Tx = __uint_as_float(static_cast<uint32_t>(__ldg(p.T + trow * V + x)) << 16);
-                    }
+                    if (warp == 0) set_device_error(&p.hdr->status, SVD_ERR_TOKEN_RANGE);
+                    xv = -1;
+                } else if (STOCH) {
+                    Dx = __uint_as_float(static_cast<uint32_t>(__ldg(p.D + drow * V + xv)) << 16);
+                    Tx = __uint_as_float(static_cast<uint32_t>(__ldg(p.T + trow * V + xv)) << 16);
                 }
             }
-            c.g.x = x;
-            c.g.Dx = Dx;
-            c.g.Tx = Tx;
+            xv = __shfl_sync(0xffffffffu, xv, 0);
+            Dx = __shfl_sync(0xffffffffu, Dx, 0);
+            Tx = __shfl_sync(0xffffffffu, Tx, 0);
+            x = xv < 0 ? kNone : static_cast<uint32_t>(xv);
         }
 
-        // -------------------------------------------------------- pass A: stream the slice
-        float e[NV][8];
-        float ref[NV];
-        float RD = kNegInf, sD = 0.f, RT = kNegInf, sT = 0.f;
-        uint4 bestDraw = make_uint4(0, 0, 0, 0), bestTraw = make_uint4(0, 0, 0, 0);
-        int bestDj = -1, bestTj = -1;
-        bool timed_out = false;
+        // -------------------------------------------------------- pass A
+        // the warp's run of D and T in its staging buffer: bulk copies (aligned rows) or plain
+        // loads (elements past the row end read as -inf)
+        if (ALIGNED) {
+            if (!wait_dead && !mbar_wait_bounded(&full[warp], phase, p.wait_limit_ns)) {
+                wait_dead = true;
+                set_device_error(&p.hdr->status, SVD_ERR_TIMEOUT);
+            }
+        } else {
+            // plain loads; elements past the row end read as the sentinel
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int lv = j * 32 + lane;
+                if (lv < wcnt) {
+                    uint16_t dv[8], tv[8];
+                    const int base = v0 + (wv0 + lv) * 8;
+#pragma unroll
+                    for (int l = 0; l < 8; ++l) {
+                        const bool ok = base + l < V && (wv0 + lv) * 8 + l < len;
+                        dv[l] = ok && isRow ? __ldg(p.D + drow * V + base + l) : (uint16_t)0xFF7Fu;
+                        tv[l] = ok ? __ldg(p.T + trow * V + base + l) : (uint16_t)0xFF7Fu;
+                    }
+                    myD[lv] = make_uint4(dv[0] | (uint32_t(dv[1]) << 16), dv[2] | (uint32_t(dv[3]) << 16),
+                                         dv[4] | (uint32_t(dv[5]) << 16), dv[6] | (uint32_t(dv[7]) << 16));
+                    myT[lv] = make_uint4(tv[0] | (uint32_t(tv[1]) << 16), tv[2] | (uint32_t(tv[3]) << 16),
+                                         tv[4] | (uint32_t(tv[5]) << 16), tv[6] | (uint32_t(tv[7]) << 16));
+                }
+            }
+            __syncwarp();
+        }
+        // pre-pass: this thread's maxima (exact bf16 compares) and the first vector holding each
+        float RD = kNegInf, RT = kNegInf;
+        int bjD = 0, bjT = 0;
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
-            if (p.aligned && !wait_dead) {
-                if (!mbar_wait_bounded(&full[j], phase, p.wait_limit_ns)) {
-                    timed_out = true;
-                    wait_dead = true;
-                }
+            const float mT = max8_bf16(myT[j * 32 + lane]);
+            const bool upT = mT > RT;
+            RT = upT ? mT : RT;
+            bjT = upT ? j : bjT;
+            if (isRow) {
+                const float mD = max8_bf16(myD[j * 32 + lane]);
+                const bool upD = mD > RD;
+                RD = upD ? mD : RD;
+                bjD = upD ? j : bjD;
             }
-            const int vi = j * NT + t;
-            const bool valid = vi < nvec;
+        }
+        // argmax candidates: the first element equal to the thread maximum in that vector
+        uint32_t candD = kNone, candT = kNone;
+        {
+            float xv[8];
+            unpack8(myT[bjT * 32 + lane], xv);
+            int l = 0;
+            while (l < 7 && xv[l] != RT) ++l;
+            candT = static_cast<uint32_t>(v0 + (wv0 + bjT * 32 + lane) * 8 + l);
+        }
+        if (rowVerify && p.draft == nullptr) {
+            float xv[8];
+            unpack8(myD[bjD * 32 + lane], xv);
+            int l = 0;
+            while (l < 7 && xv[l] != RD) ++l;
+            candD = static_cast<uint32_t>(v0 + (wv0 + bjD * 32 + lane) * 8 + l);
+        }
+        // main pass: exp relative to the thread maxima (no rescaling), online reverse-KL moment;
+        // straight-line over all rounds (sentinel vectors contribute exact zeros)
+        float e[NV][8];
+        float emax[NV];
+        float sD = 0.f, sDd = 0.f, sT = 0.f, dmax = kNegInf;
+        // (a thread holding sentinels only keeps a zero reference: its exps are exact zeros)
+        const float AD = RD > -1e38f ? RD * k2 : 0.f, AT = RT > -1e38f ? RT * k2 : 0.f;
 #pragma unroll
-            for (int l = 0; l < 8; ++l) e[j][l] = 0.f;
-            ref[j] = 0.f;
-            if (valid) {
-                uint4 rd = make_uint4(0, 0, 0, 0), rt;
-                uint32_t validmask = 0xffu;
-                if (p.aligned) {
-                    if (isRow) rd = stageD[j * NT + t];
-                    rt = stageT[j * NT + t];
-                } else {
-                    // plain loads; elements past the row end read as -inf
-                    uint16_t dv[8], tv[8];
-                    const int base = v0 + vi * 8;
+        for (int j = 0; j < NV; ++j) {
+            const int lv = j * 32 + lane;
+            emax[j] = 0.f;
+            if (!need_lse) {
 #pragma unroll
-                    for (int l = 0; l < 8; ++l) {
-                        const bool ok = base + l < V && vi * 8 + l < len;
-                        if (!ok) validmask &= ~(1u << l);
-                        dv[l] = ok && isRow ? __ldg(p.D + drow * V + base + l) : (uint16_t)0xFF80u;
-                        tv[l] = ok ? __ldg(p.T + trow * V + base + l) : (uint16_t)0xFF80u;
-                    }
-                    rd = make_uint4(dv[0] | (uint32_t(dv[1]) << 16), dv[2] | (uint32_t(dv[3]) << 16),
-                                    dv[4] | (uint32_t(dv[5]) << 16), dv[6] | (uint32_t(dv[7]) << 16));
-                    rt = make_uint4(tv[0] | (uint32_t(tv[1]) << 16), tv[2] | (uint32_t(tv[3]) << 16),
-                                    tv[4] | (uint32_t(tv[5]) << 16), tv[6] | (uint32_t(tv[7]) << 16));
+                for (int l = 0; l < 8; ++l) e[j][l] = 0.f;
+                continue;
+            }
+            float xt[8], et[8];
+            unpack8(myT[lv], xt);
+#pragma unroll
+            for (int l = 0; l < 8; ++l) et[l] = fast_exp2(fmaf(xt[l], k2, -AT));
+            sT += sum8(et);
+            if (isRow) {
+                float xd[8], dd[8];
+                unpack8(myD[lv], xd);
+#pragma unroll
+                for (int l = 0; l < 8; ++l) {
+                    e[j][l] = fast_exp2(fmaf(xd[l], k2, -AD));
+                    dd[l] = xd[l] - xt[l];
                 }
-                float xt[8];
-                unpack8(rt, xt);
-                const float mT = max8_bf16(rt);
-                if (mT > RT) {
-                    if (need_lse) sT *= fast_exp2((RT - mT) * k2);
-                    RT = mT;
-                    bestTraw = rt;
-                    bestTj = j;
+                sD += sum8(e[j]);
+                float a0 = e[j][0] * dd[0], a1 = e[j][1] * dd[1];
+                a0 = fmaf(e[j][2], dd[2], a0); a1 = fmaf(e[j][3], dd[3], a1);
+                a0 = fmaf(e[j][4], dd[4], a0); a1 = fmaf(e[j][5], dd[5], a1);
+                a0 = fmaf(e[j][6], dd[6], a0); a1 = fmaf(e[j][7], dd[7], a1);
+                sDd += a0 + a1;
+                if (DISTILL) {
+                    dmax = fmaxf(dmax, max8f(dd));
+                    emax[j] = max8f(e[j]);
                 }
-                if (isRow) {
-                    float xd[8];
-                    unpack8(rd, xd);
-                    const float mD = max8_bf16(rd);
-                    if (mD > RD) {
-                        if (need_lse) sD *= fast_exp2((RD - mD) * k2);
-                        RD = mD;
-                        bestDraw = rd;
-                        bestDj = j;
-                    }
-                    if (need_lse) {
-                        const float AD = RD * k2, AT = RT * k2;
-                        ref[j] = RD;
+                dplane[(2 * j) * NT + t] = make_float4(dd[0], dd[1], dd[2], dd[3]);
+                dplane[(2 * j + 1) * NT + t] = make_float4(dd[4], dd[5], dd[6], dd[7]);
+            } else {
 #pragma unroll
-                        for (int l = 0; l < 8; ++l) {
-                            const float ed = fast_exp2(fmaf(xd[l], k2, -AD));
-                            e[j][l] = ed;
-                            sD += ed;
-                            sT += fast_exp2(fmaf(xt[l], k2, -AT));
-                        }
-                        float dd[8];
-#pragma unroll
-                        for (int l = 0; l < 8; ++l)
-                            dd[l] = ((validmask >> l) & 1u) ? xd[l] - xt[l] : 0.f;
-                        dplane[(2 * j) * NT + t] = make_float4(dd[0], dd[1], dd[2], dd[3]);
-                        dplane[(2 * j + 1) * NT + t] = make_float4(dd[4], dd[5], dd[6], dd[7]);
-                    }
-                } else if (need_lse) {
-                    const float AT = RT * k2;
-                    ref[j] = RT;
-#pragma unroll
-                    for (int l = 0; l < 8; ++l) {
-                        const float et = fast_exp2(fmaf(xt[l], k2, -AT));
-                        e[j][l] = et;
-                        sT += et;
-                    }
-                }
+                for (int l = 0; l < 8; ++l) e[j][l] = et[l];
             }
         }
         phase ^= 1u;
-        if (timed_out) set_device_error(&p.hdr->status, SVD_ERR_TIMEOUT);
+        __syncwarp();
+        // this warp's staging is free: start the next item's copies now
+        if (ALIGNED && lane == 0 && nxt.kind != kItemNone) issue_loads(nxt);
 
-        // per-thread partials -> warp (own maxima stay per-thread for the lazy argmax)
-        float wmD = RD, wsD = sD, wmT = RT, wsT = sT;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, wmD, o);
-            const float s2 = __shfl_xor_sync(0xffffffffu, wsD, o);
-            const float m3 = __shfl_xor_sync(0xffffffffu, wmT, o);
-            const float s3 = __shfl_xor_sync(0xffffffffu, wsT, o);
-            lse_merge(wmD, wsD, m2, s2, k2);
-            lse_merge(wmT, wsT, m3, s3, k2);
-        }
-        if (lane == 0) {
-            c.wred[warp][0] = wmD;
-            c.wred[warp][1] = wsD;
-            c.wred[warp][2] = wmT;
-            c.wred[warp][3] = wsT;
-        }
-        __syncthreads();  // staging fully consumed; warp partials visible
+        // reduction #1: warp -> CTA (local shared memory) -> cluster (one DSMEM load per rank)
         {
-            const int nk = c.nkind;
-            if (t == 0 && p.aligned && (nk == kItemRow || nk == kItemBonus))
-                issue_loads(nk, c.nb, c.ni);
+            Part1 a;
+            a.mD = RD; a.sD = sD; a.sDd = sDd; a.dmax = dmax; a.mT = RT; a.sT = sT;
+            a.pad0 = a.pad1 = 0.f;
+            const Part1 r = warp_reduce_part1(a, k2);
+            if (lane == 0) c.p1[warp] = r;
         }
+        __syncthreads();
         if (warp == 0) {
-            float m0 = kNegInf, s0 = 0.f, m1 = kNegInf, s1 = 0.f;
-            if (lane < NW) { m0 = c.wred[lane][0]; s0 = c.wred[lane][1]; m1 = c.wred[lane][2]; s1 = c.wred[lane][3]; }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float a = __shfl_xor_sync(0xffffffffu, m0, o);
-                const float bb = __shfl_xor_sync(0xffffffffu, s0, o);
-                const float cc = __shfl_xor_sync(0xffffffffu, m1, o);
-                const float d = __shfl_xor_sync(0xffffffffu, s1, o);
-                lse_merge(m0, s0, a, bb, k2);
-                lse_merge(m1, s1, cc, d, k2);
-            }
-            if (lane == 0) { c.slot.mD = m0; c.slot.sD = s0; c.slot.mT = m1; c.slot.sT = s1; }
+            const Part1 a = lane < NW ? c.p1[lane] : empty_part1();
+            const Part1 r = warp_reduce_part1(a, k2);
+            if (lane == 0) c.cta1 = r;
         }
         cluster_sync();  // #1
 
-        // ---------------------------------------------------- row statistics (every rank)
-        if (warp == 0) {
-            float m0 = kNegInf, s0 = 0.f, m1 = kNegInf, s1 = 0.f;
-            if (lane < static_cast<int>(CL)) {
-                const uint32_t a = dsmem_map(&c.slot, lane);
-                m0 = dsmem_ld_f32(a + offsetof(Slot, mD));
-                s0 = dsmem_ld_f32(a + offsetof(Slot, sD));
-                m1 = dsmem_ld_f32(a + offsetof(Slot, mT));
-                s1 = dsmem_ld_f32(a + offsetof(Slot, sT));
+        // ------------------------------------------------ row statistics (every warp)
+        float MD, MT, lseD = kQNaN, lseT = kQNaN, L2D = 0.f, L2T = 0.f, dl = 0.f, rkl = 0.f, smax = 0.f;
+        {
+            Part1 a = empty_part1();
+            if (lane < CL) {
+                const uint32_t ad = dsmem_map(&c.cta1, lane);
+                float v[4], u[4];
+                dsmem_ld4(ad, v);
+                dsmem_ld4(ad + 16, u);
+                a.mD = v[0]; a.sD = v[1]; a.sDd = v[2]; a.dmax = v[3]; a.mT = u[0]; a.sT = u[1];
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float a = __shfl_xor_sync(0xffffffffu, m0, o);
-                const float bb = __shfl_xor_sync(0xffffffffu, s0, o);
-                const float cc = __shfl_xor_sync(0xffffffffu, m1, o);
-                const float d = __shfl_xor_sync(0xffffffffu, s1, o);
-                lse_merge(m0, s0, a, bb, k2);
-                lse_merge(m1, s1, cc, d, k2);
-            }
-            if (lane == 0) {
-                RowG& g = c.g;
-                g.MD = m0;
-                g.MT = m1;
-                if (need_lse) {
-                    g.lseD = isRow ? m0 * itau + logf(s0) : __int_as_float(0x7fc00000);
-                    g.lseT = m1 * itau + logf(s1);
-                    g.L2D = g.lseD * kLog2e;
-                    g.L2T = g.lseT * kLog2e;
-                    g.dl = g.lseD - g.lseT;
-                } else {
-                    g.lseD = g.lseT = __int_as_float(0x7fc00000);
-                    g.L2D = g.L2T = g.dl = 0.f;
+            const Part1 r = warp_reduce_part1(a, k2);   // identical in every lane, warp and rank
+            MD = r.mD;
+            MT = r.mT;
+            if (need_lse) {
+                if (isRow) lseD = r.mD * itau + logf(r.sD);
+                lseT = r.mT * itau + logf(r.sT);
+                L2D = lseD * kLog2e;
+                L2T = lseT * kLog2e;
+                dl = lseD - lseT;
+                if (isRow) {
+                    rkl = (r.sDd / r.sD) * itau - dl;   // sum_v q_v (log q_v - log p_v)
+                    smax = r.dmax * itau - dl;          // largest log q_v - log p_v
                 }
-                g.ratio = __int_as_float(0x7fc00000);
-                g.acc = 0;
-                g.do_sample = 0;
-                g.attempt_p = 0;
-                g.u0 = g.u1 = 0.f;
-                if (STOCH) {
-                    const PhiloxOut ph = philox_words(p.seed, p.step, static_cast<uint32_t>(b),
-                                                      static_cast<uint32_t>(i));
-                    g.u0 = uniform24(ph.w[0]);
-                    g.u1 = uniform24(ph.w[1]);
-                    if (rowVerify) {
-                        if (g.x != kNone) {
-                            g.ratio = fast_exp2((g.dl - (g.Dx - g.Tx) * itau) * kLog2e);
-                            g.acc = g.u0 < fminf(1.f, g.ratio) ? 1 : 0;
-                        } else {
-                            g.ratio = 0.f;
-                            g.acc = 0;
-                        }
-                        g.do_sample = g.acc ? 0 : 1;
-                    } else if (!isRow) {
-                        g.do_sample = 1;  // bonus row: sample from p
+            }
+        }
+        // rank 0 completes the previous row's record while the rest of the cluster works
+        if (pending && rank == 0 && warp == NW - 1) finish_record();
+        pending = false;
+
+        // stochastic decision (every warp computes the same value)
+        float ratio = kQNaN, u1 = 0.f;
+        int acc = 0, do_sample = 0;
+        if (STOCH) {
+            const PhiloxOut ph = philox_words(p.seed, p.step, static_cast<uint32_t>(b),
+                                              static_cast<uint32_t>(i));
+            const float u0 = uniform24(ph.w[0]);
+            u1 = uniform24(ph.w[1]);
+            if (rowVerify) {
+                if (x != kNone) {
+                    ratio = fast_exp2((dl - (Dx - Tx) * itau) * kLog2e);
+                    acc = u0 < fminf(1.f, ratio) ? 1 : 0;
+                } else {
+                    ratio = 0.f;
+                    acc = 0;
+                }
+                do_sample = acc ? 0 : 1;
+            } else if (!isRow) {
+                do_sample = 1;  // bonus row: sample from p
+            }
+        }
+
+        // lazy argmax: only the threads holding the row maximum offer their candidate
+        Deposit* dep0 = &c.dep[par];
+        if (candD != kNone && RD == MD) dsmem_min_u32(dsmem_map(&dep0->argD, 0), candD);
+        if (candT != kNone && RT == MT) dsmem_min_u32(dsmem_map(&dep0->argT, 0), candT);
+
+        // -------------------------------------------------------- pass B
+        // q_v = e_v * f with one factor per thread; only entries with q_v > c / s_max can be
+        // clipped (d_v = q_v s_v <= q_v s_max), so the exact test runs on those vectors alone
+        const float fD = isRow ? fast_exp2(AD - L2D) : 0.f;
+        const float fT = fast_exp2(AT - L2T);
+        float clip_d = 0.f, clip_q = 0.f, n_clip = 0.f;
+        uint32_t clipmask = 0;
+        const float cc = p.clip_c;
+        if (DISTILL && isRow && isfinite(cc) && smax > 0.f) {
+            const float qthr = (cc / smax) * 0.9999f;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                if (emax[j] * fD > qthr) {
+                    clipmask |= 1u << j;
+                    const float4 lo = dplane[(2 * j) * NT + t];
+                    const float4 hi = dplane[(2 * j + 1) * NT + t];
+                    const float dd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                    for (int l = 0; l < 8; ++l) {
+                        const float q = elem_q(e[j][l], fD);
+                        const float d = elem_d(q, elem_s(dd[l], itau, dl));
+                        if (d > cc) { clip_d += d; clip_q += q; n_clip += 1.f; }
                     }
                 }
             }
         }
-        __syncthreads();
-
-        // lazy argmax: only the threads that hold the row maximum inspect their best vector
-        {
-            const RowG& g = c.g;
-            const uint32_t rank0 = 0;
-            if (rowVerify && p.draft == nullptr && bestDj >= 0 && RD == g.MD) {
-                float xd[8];
-                unpack8(bestDraw, xd);
-                int l = 0;
-                while (l < 7 && xd[l] != g.MD) ++l;
-                dsmem_min_u32(dsmem_map(&c.slot.argD, rank0),
-                              static_cast<uint32_t>(v0 + (bestDj * NT + t) * 8 + l));
-            }
-            if (bestTj >= 0 && RT == g.MT) {
-                float xt[8];
-                unpack8(bestTraw, xt);
-                int l = 0;
-                while (l < 7 && xt[l] != g.MT) ++l;
-                dsmem_min_u32(dsmem_map(&c.slot.argT, rank0),
-                              static_cast<uint32_t>(v0 + (bestTj * NT + t) * 8 + l));
-            }
-        }
-
-        // -------------------------------------------------------- pass B
-        float sum_d = 0.f, clip_d = 0.f, clip_q = 0.f, n_clip = 0.f;
-        uint32_t clipmask = 0;
-        unsigned long long vmass[NV];
+        unsigned long long vmass[NV], vpre[NV];
 #pragma unroll
-        for (int j = 0; j < NV; ++j) vmass[j] = 0ull;
-        const bool has_clip = DISTILL && isRow && isfinite(p.clip_c);
-        const bool do_sample = STOCH && c.g.do_sample;
-        if ((DISTILL && isRow) || do_sample) {
-            const RowG& g = c.g;
-            const float dl = g.dl, cc = p.clip_c;
+        for (int j = 0; j < NV; ++j) { vmass[j] = 0ull; vpre[j] = 0ull; }
+        if (STOCH && do_sample) {
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
-                const int vi = j * NT + t;
-                if (vi < nvec) {
+                {
+                    unsigned long long ms = 0ull;
                     if (isRow) {
-                        const float f = fast_exp2(ref[j] * k2 - g.L2D);
                         const float4 lo = dplane[(2 * j) * NT + t];
                         const float4 hi = dplane[(2 * j + 1) * NT + t];
                         const float dd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                        float vmax = kNegInf;
-                        unsigned long long ms = 0ull;
 #pragma unroll
                         for (int l = 0; l < 8; ++l) {
-                            const float q = elem_q(e[j][l], f);
-                            const float s = elem_s(dd[l], itau, dl);
-                            if (DISTILL) {
-                                const float d = elem_d(q, s);
-                                sum_d += d;
-                                vmax = fmaxf(vmax, d);
-                            }
-                            if (STOCH && do_sample)
-                                ms += to_fixed(fmaxf(__fsub_rn(elem_p(q, s), q), 0.f));
+                            const float q = elem_q(e[j][l], fD);
+                            ms += to_fixed(fmaxf(__fsub_rn(elem_p(q, elem_s(dd[l], itau, dl)), q), 0.f));
                         }
-                        if (STOCH) vmass[j] = ms;
-                        if (has_clip && vmax > cc) {
-                            clipmask |= 1u << j;
+                    } else {
 #pragma unroll
-                            for (int l = 0; l < 8; ++l) {
-                                const float q = elem_q(e[j][l], f);
-                                const float d = elem_d(q, elem_s(dd[l], itau, dl));
-                                if (d > cc) { clip_d += d; clip_q += q; n_clip += 1.f; }
-                            }
-                        }
-                    } else if (STOCH) {
-                        // bonus row: masses of p itself
-                        const float f = fast_exp2(ref[j] * k2 - g.L2T);
-                        unsigned long long ms = 0ull;
-#pragma unroll
-                        for (int l = 0; l < 8; ++l) ms += to_fixed(elem_q(e[j][l], f));
-                        vmass[j] = ms;
+                        for (int l = 0; l < 8; ++l) ms += to_fixed(elem_q(e[j][l], fT));
                     }
+                    vmass[j] = ms;
                 }
             }
         }
-
-        // exclusive prefix of the sample masses in (round, thread) order; CTA total
-        unsigned long long vpre[NV];
-#pragma unroll
-        for (int j = 0; j < NV; ++j) vpre[j] = 0ull;
-        unsigned long long cta_mass = 0ull;
+        // warp prefix of the sample masses in id order (round-major, then lane)
+        unsigned long long wmass = 0ull;
         if (STOCH && do_sample) {
-            unsigned long long carry = 0ull;
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
                 unsigned long long incl = vmass[j];
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += y;
-                }
-                if (lane == 31) c.wmass[warp] = incl;
-                __syncthreads();
-                unsigned long long woff = 0ull, tot = 0ull;
-                for (int q = 0; q < NW; ++q) {
-                    const unsigned long long v = c.wmass[q];
-                    if (q < warp) woff += v;
-                    tot += v;
-                }
-                vpre[j] = carry + woff + incl - vmass[j];
-                carry += tot;
-                __syncthreads();
+                warp_inclusive_scan_u64(incl);
+                vpre[j] = wmass + incl - vmass[j];
+                wmass += __shfl_sync(0xffffffffu, incl, 31);
             }
-            cta_mass = carry;
         }
-
-        // CTA partials of pass B -> slot
+        // reduction #2: warp -> CTA (fixed order) -> cluster
         if (DISTILL && isRow) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                sum_d += __shfl_xor_sync(0xffffffffu, sum_d, o);
-                clip_d += __shfl_xor_sync(0xffffffffu, clip_d, o);
-                clip_q += __shfl_xor_sync(0xffffffffu, clip_q, o);
-                n_clip += __shfl_xor_sync(0xffffffffu, n_clip, o);
-            }
-            if (lane == 0) {
-                c.wred[warp][0] = sum_d;
-                c.wred[warp][1] = clip_d;
-                c.wred[warp][2] = clip_q;
-                c.wred[warp][3] = n_clip;
-            }
+            clip_d = warp_sum(clip_d);
+            clip_q = warp_sum(clip_q);
+            n_clip = warp_sum(n_clip);
+        }
+        if (lane == 0) {
+            Part2 q2;
+            q2.clip_d = clip_d; q2.clip_q = clip_q; q2.n_clip = n_clip; q2.pad0 = 0.f;
+            q2.mass = wmass;
+            q2.pad1 = 0ull;
+            c.p2[warp] = q2;
         }
         __syncthreads();
-        if (t == 0) {
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            if (DISTILL && isRow) {
-                for (int q = 0; q < NW; ++q) {
-                    a0 += c.wred[q][0];
-                    a1 += c.wred[q][1];
-                    a2 += c.wred[q][2];
-                    a3 += c.wred[q][3];
-                }
+        if (warp == 0) {
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+            unsigned long long m = 0ull;
+            if (lane < NW) {
+                const Part2 q = c.p2[lane];
+                a0 = q.clip_d; a1 = q.clip_q; a2 = q.n_clip; m = q.mass;
             }
-            c.slot.sum_d = a0;
-            c.slot.clip_d = a1;
-            c.slot.clip_q = a2;
-            c.slot.n_clip = a3;
-            c.slot.mass = cta_mass;
+            unsigned long long incl = m;
+            warp_inclusive_scan_u64(incl);
+            if (lane < NW) c.wpre[lane] = incl - m;
+            a0 = warp_sum(a0);
+            a1 = warp_sum(a1);
+            a2 = warp_sum(a2);
+            const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
+            if (lane == 0) {
+                Part2 q2;
+                q2.clip_d = a0; q2.clip_q = a1; q2.n_clip = a2; q2.pad0 = 0.f;
+                q2.mass = tot;
+                q2.pad1 = 0ull;
+                c.cta2 = q2;
+            }
         }
         cluster_sync();  // #2
 
-        // ---------------------------------------------------- row results (every rank)
-        if (warp == 0) {
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            unsigned long long mass = 0ull, before = 0ull;
-            if (lane < static_cast<int>(CL)) {
-                const uint32_t a = dsmem_map(&c.slot, lane);
-                a0 = dsmem_ld_f32(a + offsetof(Slot, sum_d));
-                a1 = dsmem_ld_f32(a + offsetof(Slot, clip_d));
-                a2 = dsmem_ld_f32(a + offsetof(Slot, clip_q));
-                a3 = dsmem_ld_f32(a + offsetof(Slot, n_clip));
-                const uint32_t lo = dsmem_ld_u32(a + offsetof(Slot, mass));
-                const uint32_t hi = dsmem_ld_u32(a + offsetof(Slot, mass) + 4);
-                mass = (static_cast<unsigned long long>(hi) << 32) | lo;
+        // ------------------------------------------------ row results (every warp)
+        float kc = 0.f, P = 0.f, Q = 0.f, Pc = 0.f, hardc = 0.f;
+        unsigned long long R = 0ull, before = 0ull;
+        {
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+            unsigned long long m = 0ull;
+            if (lane < CL) {
+                const uint32_t a = dsmem_map(&c.cta2, lane);
+                float v[4];
+                dsmem_ld4(a, v);
+                a0 = v[0]; a1 = v[1]; a2 = v[2];
+                m = dsmem_ld_u64(a + offsetof(Part2, mass));
             }
-            // fixed-order sums over ranks (lane order), identical on every rank
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-            unsigned long long R = 0ull;
-            for (int r = 0; r < static_cast<int>(CL); ++r) {
-                s0 += __shfl_sync(0xffffffffu, a0, r);
-                s1 += __shfl_sync(0xffffffffu, a1, r);
-                s2 += __shfl_sync(0xffffffffu, a2, r);
-                s3 += __shfl_sync(0xffffffffu, a3, r);
-                const unsigned long long mr = __shfl_sync(0xffffffffu, mass, r);
-                if (r < static_cast<int>(rank)) before += mr;
-                R += mr;
+            R = m;
+            before = (lane < static_cast<int>(rank)) ? m : 0ull;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                R += __shfl_xor_sync(0xffffffffu, R, o);
+                before += __shfl_xor_sync(0xffffffffu, before, o);
             }
-            if (lane == 0) {
-                RowG& g = c.g;
-                const uint32_t a = dsmem_map(&c.slot, 0);
-                const uint32_t argD = dsmem_ld_u32(a + offsetof(Slot, argD));
-                const uint32_t argT = dsmem_ld_u32(a + offsetof(Slot, argT));
-                g.y = argT;
-                if (isRow && p.draft == nullptr) g.x = argD;
-                if (rowVerify && !STOCH) g.acc = (g.x == g.y) ? 1 : 0;
-                g.R = R;
-                g.off = before;
-                g.tgt = scale_mass(R, static_cast<uint32_t>(g.u1 * 16777216.0f));
-                g.sum_d = s0;
-                g.clip_d = s1;
-                g.n_clip = s3;
-                if (DISTILL && isRow) {
-                    // S = sum over unclipped entries of q (s + 1) = (sum_d - clip_d) + (1 - clip_q)
-                    const float S = (s0 - s1) + (1.f - s2);
-                    const float lam = p.lambda, pre = p.grad_scale * itau;
-                    g.P = pre * (lam + (1.f - lam) * (1.f - S - g.dl));
-                    g.Q = pre * (1.f - lam) * itau;
-                    g.Pc = pre * (lam - (1.f - lam) * S);
-                    g.hardc = pre * lam;
-                }
-                if (STOCH && g.do_sample && R == 0ull) g.attempt_p = 1;
+            before += c.wpre[warp];
+            if (DISTILL && isRow) {
+                a0 = warp_sum(a0);
+                a1 = warp_sum(a1);
+                a2 = warp_sum(a2);
+                // S = sum over unclipped entries of q (s + 1) = (rkl - clip_d) + (1 - clip_q)
+                const float S = (rkl - a0) + (1.f - a1);
+                kc = isfinite(cc) ? (rkl - a0) + cc * a2 : rkl;
+                const float lam = p.lambda, pre = p.grad_scale * itau;
+                P = pre * (lam + (1.f - lam) * (1.f - S - dl));
+                Q = pre * (1.f - lam) * itau;
+                Pc = pre * (lam - (1.f - lam) * S);
+                hardc = pre * lam;
             }
         }
-        __syncthreads();
+        uint32_t y = kNone;
+        {
+            const uint32_t a = dsmem_map(dep0, 0);
+            uint32_t yv = 0, xv = 0;
+            if (lane == 0) {
+                yv = dsmem_ld_u32(a + offsetof(Deposit, argT));
+                if (rowVerify && p.draft == nullptr) xv = dsmem_ld_u32(a + offsetof(Deposit, argD));
+            }
+            y = __shfl_sync(0xffffffffu, yv, 0);
+            if (rowVerify && p.draft == nullptr) x = __shfl_sync(0xffffffffu, xv, 0);
+        }
+        if (rowVerify && !STOCH) acc = (x == y) ? 1 : 0;
 
-        // stochastic fallback: residual mass zero -> sample from p (rare; extra reduction)
-        if (STOCH && do_sample && c.g.attempt_p) {
-            const RowG& g = c.g;
+        // stochastic fallback: residual mass zero -> sample from p (rare; one more reduction)
+        bool use_p = false;
+        if (STOCH && do_sample && R == 0ull && isRow) {
+            use_p = true;
+            wmass = 0ull;
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
                 vmass[j] = 0ull;
-                const int vi = j * NT + t;
-                if (vi < nvec) {
-                    const float f = fast_exp2(ref[j] * k2 - g.L2D);
+                if (j * 32 + lane < wcnt) {
                     const float4 lo = dplane[(2 * j) * NT + t];
                     const float4 hi = dplane[(2 * j + 1) * NT + t];
                     const float dd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
                     unsigned long long ms = 0ull;
 #pragma unroll
-                    for (int l = 0; l < 8; ++l) {
-                        const float q = elem_q(e[j][l], f);
-                        ms += to_fixed(elem_p(q, elem_s(dd[l], itau, g.dl)));
-                    }
+                    for (int l = 0; l < 8; ++l)
+                        ms += to_fixed(elem_p(elem_q(e[j][l], fD), elem_s(dd[l], itau, dl)));
                     vmass[j] = ms;
                 }
-            }
-            unsigned long long carry = 0ull;
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
                 unsigned long long incl = vmass[j];
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += y;
-                }
-                if (lane == 31) c.wmass[warp] = incl;
-                __syncthreads();
-                unsigned long long woff = 0ull, tot = 0ull;
-                for (int q = 0; q < NW; ++q) {
-                    const unsigned long long v = c.wmass[q];
-                    if (q < warp) woff += v;
-                    tot += v;
-                }
-                vpre[j] = carry + woff + incl - vmass[j];
-                carry += tot;
-                __syncthreads();
+                warp_inclusive_scan_u64(incl);
+                vpre[j] = wmass + incl - vmass[j];
+                wmass += __shfl_sync(0xffffffffu, incl, 31);
             }
-            if (t == 0) c.slot.mass2 = carry;
-            cluster_sync();
-            if (t == 0) {
-                unsigned long long R = 0ull, before = 0ull;
-                for (int r = 0; r < static_cast<int>(CL); ++r) {
-                    const uint32_t a = dsmem_map(&c.slot, r);
-                    const uint32_t lo = dsmem_ld_u32(a + offsetof(Slot, mass2));
-                    const uint32_t hi = dsmem_ld_u32(a + offsetof(Slot, mass2) + 4);
-                    const unsigned long long mr = (static_cast<unsigned long long>(hi) << 32) | lo;
-                    if (r < static_cast<int>(rank)) before += mr;
-                    R += mr;
-                }
-                c.g.R = R;
-                c.g.off = before;
-                c.g.tgt = scale_mass(R, static_cast<uint32_t>(c.g.u1 * 16777216.0f));
-            }
+            if (lane == 0) c.p2[warp].mass = wmass;
             __syncthreads();
+            if (warp == 0) {
+                const unsigned long long m = lane < NW ? c.p2[lane].mass : 0ull;
+                unsigned long long incl = m;
+                warp_inclusive_scan_u64(incl);
+                if (lane < NW) c.wpre[lane] = incl - m;
+                const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
+                if (lane == 0) c.cta3.mass = tot;
+            }
+            cluster_sync();
+            {
+                const unsigned long long m =
+                    lane < CL ? dsmem_ld_u64(dsmem_map(&c.cta3, lane) + offsetof(Part2, mass)) : 0ull;
+                R = m;
+                before = (lane < static_cast<int>(rank)) ? m : 0ull;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    R += __shfl_xor_sync(0xffffffffu, R, o);
+                    before += __shfl_xor_sync(0xffffffffu, before, o);
+                }
+                before += c.wpre[warp];
+            }
         }
 
         // -------------------------------------------------------- sample search
-        if (STOCH && do_sample && c.g.R > 0ull) {
-            const RowG& g = c.g;
-            const bool use_p = g.attempt_p != 0;
+        if (STOCH && do_sample && R > 0ull) {
+            const unsigned long long tgt = scale_mass(R, static_cast<uint32_t>(u1 * 16777216.0f));
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
-                const int vi = j * NT + t;
-                const unsigned long long lo = g.off + vpre[j];
-                if (vi < nvec && vmass[j] > 0ull && lo <= g.tgt && g.tgt - lo < vmass[j]) {
+                const unsigned long long lo = before + vpre[j];
+                if (j * 32 + lane < wcnt && vmass[j] > 0ull && lo <= tgt && tgt - lo < vmass[j]) {
                     // the sample point lies in this vector: walk its 8 masses in id order
-                    const unsigned long long rel = g.tgt - lo;
+                    const unsigned long long rel = tgt - lo;
                     unsigned long long cum = 0ull;
                     int pick = -1;
                     if (isRow) {
-                        const float f = fast_exp2(ref[j] * k2 - g.L2D);
                         const float4 a = dplane[(2 * j) * NT + t];
                         const float4 bq = dplane[(2 * j + 1) * NT + t];
                         const float dd[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
                         for (int l = 0; l < 8; ++l) {
-                            const float q = elem_q(e[j][l], f);
-                            const float pv = elem_p(q, elem_s(dd[l], itau, g.dl));
+                            const float q = elem_q(e[j][l], fD);
+                            const float pv = elem_p(q, elem_s(dd[l], itau, dl));
                             cum += use_p ? to_fixed(pv) : to_fixed(fmaxf(__fsub_rn(pv, q), 0.f));
                             if (pick < 0 && cum > rel) pick = l;
                         }
                     } else {
-                        const float f = fast_exp2(ref[j] * k2 - g.L2T);
 #pragma unroll
                         for (int l = 0; l < 8; ++l) {
-                            cum += to_fixed(elem_q(e[j][l], f));
+                            cum += to_fixed(elem_q(e[j][l], fT));
                             if (pick < 0 && cum > rel) pick = l;
                         }
                     }
                     if (pick < 0) pick = 7;
-                    dsmem_min_u32(dsmem_map(&c.slot.tok, 0), static_cast<uint32_t>(v0 + vi * 8 + pick));
+                    dsmem_min_u32(dsmem_map(&dep0->tok, 0),
+                                  static_cast<uint32_t>(v0 + (wv0 + j * 32 + lane) * 8 + pick));
                 }
             }
         }
 
         // -------------------------------------------------------- pass C: gradient row
         if (DISTILL && isRow) {
-            const RowG& g = c.g;
-            const float dl = g.dl, cc = p.clip_c;
-            const uint32_t y = g.y;
+            const float Pj = fD * P, Qj = fD * Q;
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
-                const int vi = j * NT + t;
-                if (vi < nvec) {
-                    const float f = fast_exp2(ref[j] * k2 - g.L2D);
-                    const float Pj = f * g.P, Qj = f * g.Q;
-                    const float4 lo = dplane[(2 * j) * NT + t];
-                    const float4 hi = dplane[(2 * j + 1) * NT + t];
-                    const float dd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                    float gv[8];
+                const int lv = j * 32 + lane;
+                const float4 lo = dplane[(2 * j) * NT + t];
+                const float4 hi = dplane[(2 * j + 1) * NT + t];
+                const float dd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                float gv[8];
 #pragma unroll
-                    for (int l = 0; l < 8; ++l) gv[l] = e[j][l] * fmaf(Qj, dd[l], Pj);
-                    if (clipmask & (1u << j)) {
+                for (int l = 0; l < 8; ++l) gv[l] = e[j][l] * fmaf(Qj, dd[l], Pj);
+                if (clipmask & (1u << j)) {
 #pragma unroll
-                        for (int l = 0; l < 8; ++l) {
-                            const float q = elem_q(e[j][l], f);
-                            const float d = elem_d(q, elem_s(dd[l], itau, dl));
-                            if (d > cc) gv[l] = q * g.Pc;
-                        }
+                    for (int l = 0; l < 8; ++l) {
+                        const float q = elem_q(e[j][l], fD);
+                        const float d = elem_d(q, elem_s(dd[l], itau, dl));
+                        if (d > cc) gv[l] = q * Pc;
                     }
-                    const int base = v0 + vi * 8;
+                }
+                if (lv < wcnt) {
+                    const int base = v0 + (wv0 + lv) * 8;
                     if (y >= static_cast<uint32_t>(base) && y < static_cast<uint32_t>(base + 8)) {
-                        const int l = static_cast<int>(y) - base;
+                        const int ly = static_cast<int>(y) - base;
                         float dy = dd[0];
 #pragma unroll
-                        for (int q = 1; q < 8; ++q) if (q == l) dy = dd[q];
+                        for (int q = 1; q < 8; ++q) if (q == ly) dy = dd[q];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) if (q == l) gv[q] -= g.hardc;
+                        for (int q = 0; q < 8; ++q) if (q == ly) gv[q] -= hardc;
                         // -log q_y = lseD - D_y / tau, with D_y = delta_y + T_y and T_y = max T
-                        dsmem_st_f32(dsmem_map(&c.slot.ce, 0), g.lseD - (dy + g.MT) * itau);
+                        dsmem_st_f32(dsmem_map(&dep0->ce, 0), lseD - (dy + MT) * itau);
                     }
-                    if (p.aligned) {
+                    if (ALIGNED) {
                         if (p.dl_fp32) {
                             float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.dlogits) + drow * V + base);
                             __stcs(o, make_float4(gv[0], gv[1], gv[2], gv[3]));
@@ -875,7 +981,7 @@ __global__ void __launch_bounds__(NT, 1) row_pass_kernel(const RowParams p) {
                     } else {
 #pragma unroll
                         for (int l = 0; l < 8; ++l) {
-                            if (base + l < V && vi * 8 + l < len) {
+                            if (base + l < V && (wv0 + lv) * 8 + l < len) {
                                 if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + base + l] = gv[l];
                                 else static_cast<uint16_t*>(p.dlogits)[drow * V + base + l] =
                                     static_cast<uint16_t>(pack_bf16x2(gv[l], 0.f) & 0xffffu);
@@ -884,142 +990,75 @@ __global__ void __launch_bounds__(NT, 1) row_pass_kernel(const RowParams p) {
                     }
                 }
             }
-        } else if (DISTILL && !isRow && i < p.k) {
+        } else if (DISTILL && !isRow && i < k) {
             // bonus row: its gradient row is zero
-            if (p.aligned) {
+            if (ALIGNED) {
                 const uint4 z = make_uint4(0, 0, 0, 0);
                 if (p.dl_fp32) {
-                    float* gp = static_cast<float*>(p.dlogits) + drow * V + v0;
-                    for (int e2 = t * 4; e2 < len; e2 += NT * 4) __stcs(reinterpret_cast<uint4*>(gp + e2), z);
+                    float* g = static_cast<float*>(p.dlogits) + drow * V + v0 + wv0 * 8;
+                    for (int e2 = lane; e2 < wcnt * 2; e2 += 32) __stcs(reinterpret_cast<uint4*>(g) + e2, z);
                 } else {
-                    uint16_t* gp = static_cast<uint16_t*>(p.dlogits) + drow * V + v0;
-                    for (int e2 = t * 8; e2 < len; e2 += NT * 8) __stcs(reinterpret_cast<uint4*>(gp + e2), z);
+                    uint16_t* g = static_cast<uint16_t*>(p.dlogits) + drow * V + v0 + wv0 * 8;
+                    for (int e2 = lane; e2 < wcnt; e2 += 32) __stcs(reinterpret_cast<uint4*>(g) + e2, z);
                 }
             } else {
-                for (int e2 = t; e2 < len; e2 += NT) {
+                const int e_end = min(len, (wv0 + wcnt) * 8);
+                for (int e2 = wv0 * 8 + lane; e2 < e_end; e2 += 32) {
                     if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + v0 + e2] = 0.f;
                     else static_cast<uint16_t*>(p.dlogits)[drow * V + v0 + e2] = 0;
                 }
             }
         }
-        cluster_sync();  // #3: deposits (token, CE) visible in rank 0
 
-        // -------------------------------------------------------- row record, ticket, scan
-        if (rank == 0 && warp == 0) {
-            int fin = 0;
-            if (lane == 0) {
-                const RowG& g = c.g;
-                svd_row_info r;
-                r.draft_token = rowVerify ? static_cast<int32_t>(g.x == kNone ? -1 : static_cast<int>(g.x)) : -1;
-                r.target_argmax = static_cast<int32_t>(g.y);
-                r.accepted = rowVerify ? g.acc : -1;
-                if (!verify) r.sample_token = -1;
-                else if (!STOCH) r.sample_token = static_cast<int32_t>(g.y);
-                else r.sample_token = (g.do_sample && c.slot.tok != kNone) ? static_cast<int32_t>(c.slot.tok) : -1;
-                r.ratio = g.ratio;
-                r.lse_draft = isRow ? g.lseD : __int_as_float(0x7fc00000);
-                r.lse_target = g.lseT;
-                float L = 0.f;
-                if (DISTILL && isRow) {
-                    const float Kc = isfinite(p.clip_c) ? (g.sum_d - g.clip_d) + p.clip_c * g.n_clip : g.sum_d;
-                    L = p.lambda * c.slot.ce + (1.f - p.lambda) * Kc;
-                    if (p.loss_rows) p.loss_rows[drow] = L;
+        // rank 0 keeps this row's values; the record is completed after the next cluster barrier
+        if (rank == 0 && warp == NW - 1 && lane == 0) {
+            Pending& pd = c.pend;
+            pd.b = b; pd.i = i; pd.kind = cur.kind;
+            pd.x = rowVerify ? (x == kNone ? -1 : static_cast<int>(x)) : -1;
+            pd.y = static_cast<int>(y);
+            pd.acc = rowVerify ? acc : -1;
+            pd.do_sample = do_sample;
+            pd.ratio = ratio;
+            pd.lseD = isRow ? lseD : kQNaN;
+            pd.lseT = lseT;
+            pd.kc = kc;
+        }
+        pending = true;
+        par ^= 1;
+        cur = nxt;
+        w = wn;
+    }
+    if (pending) {  // uniform: every rank walked the same items
+        cluster_sync();
+        if (rank == 0 && warp == NW - 1) finish_record();
+    }
+
+    // ---------------------------------------------------------------- zero-only gradient rows
+    if (DISTILL) {
+        for (int z = cid; z < p.B * k; z += ncl) {
+            const int b = z / k, i = z % k;
+            if (!zero_row_pred(k, bkv(p, b), i, verify)) continue;
+            const size_t drow = static_cast<size_t>(b) * k + i;
+            if (ALIGNED) {
+                const uint4 zz = make_uint4(0, 0, 0, 0);
+                if (p.dl_fp32) {
+                    float* g = static_cast<float*>(p.dlogits) + drow * V + v0 + wv0 * 8;
+                    for (int e = lane; e < wcnt * 2; e += 32) __stcs(reinterpret_cast<uint4*>(g) + e, zz);
+                } else {
+                    uint16_t* g = static_cast<uint16_t*>(p.dlogits) + drow * V + v0 + wv0 * 8;
+                    for (int e = lane; e < wcnt; e += 32) __stcs(reinterpret_cast<uint4*>(g) + e, zz);
                 }
-                r.loss = L;
-                p.rec[trow] = r;
-                if (p.row_info) p.row_info[trow] = r;
-                // reset the rank-0 deposit targets for the next row
-                c.slot.argD = kNone;
-                c.slot.argT = kNone;
-                c.slot.tok = kNone;
-                c.slot.ce = 0.f;
-                __threadfence();
-                const int n = get_bk(p, b);
-                const uint32_t expected = static_cast<uint32_t>(n + ((verify && n < p.kt) ? 1 : 0));
-                const uint32_t old = atomicAdd(&p.seq_ticket[b], 1u);
-                fin = (old + 1u == expected) ? 1 : 0;
-            }
-            fin = __shfl_sync(0xffffffffu, fin, 0);
-            if (fin) {
-                // ---------------- sequence b complete: acceptance scan (one lane per position)
-                __threadfence();
-                const int n = get_bk(p, b);
-                const int kt = p.kt, k = p.k;
-                svd_row_info r;
-                r.draft_token = -1; r.target_argmax = -1; r.accepted = -1; r.sample_token = -1;
-                r.ratio = r.lse_draft = r.lse_target = __int_as_float(0x7fc00000);
-                r.loss = 0.f;
-                auto is_processed = [&](int row) { return row < n || (verify && row == n && n < kt); };
-                if (lane < kt && is_processed(lane)) {
-                    const svd_row_info* src = p.rec + static_cast<size_t>(b) * kt + lane;
-                    r.draft_token = __ldcg(&src->draft_token);
-                    r.target_argmax = __ldcg(&src->target_argmax);
-                    r.accepted = __ldcg(&src->accepted);
-                    r.sample_token = __ldcg(&src->sample_token);
-                    r.loss = __ldcg(&src->loss);
-                } else if (lane < kt && p.row_info) {
-                    p.row_info[static_cast<size_t>(b) * kt + lane] = r;  // unprocessed row
-                }
-                if (kt == 33 && lane == 0 && !is_processed(32) && p.row_info) {
-                    svd_row_info u = r;
-                    u.draft_token = u.target_argmax = u.accepted = u.sample_token = -1;
-                    u.ratio = u.lse_draft = u.lse_target = __int_as_float(0x7fc00000);
-                    u.loss = 0.f;
-                    p.row_info[static_cast<size_t>(b) * kt + 32] = u;
-                }
-                if (verify) {
-                    const uint32_t accm = __ballot_sync(0xffffffffu, lane < n && r.accepted == 1);
-                    const uint32_t notacc = ~accm;
-                    int a = __ffs(notacc) - 1;
-                    if (a > n || a < 0) a = n;
-                    const int fix_row = a < n ? a : ((n < kt) ? n : -1);
-                    int fix_tok = __shfl_sync(0xffffffffu, r.sample_token, fix_row < 0 ? 0 : (fix_row & 31));
-                    if (fix_row >= 32)  // bonus row 32 (k = 32, kt = 33) has no lane of its own
-                        fix_tok = __ldcg(&p.rec[static_cast<size_t>(b) * kt + 32].sample_token);
-                    // lane q holds row q's record; slot k (= 32 at most) has no row of its own and
-                    // can only hold the correction / bonus token
-                    if (lane < k + 1) {
-                        int v = -1;
-                        if (lane < a) v = r.draft_token;
-                        else if (lane == a && fix_row >= 0) v = fix_tok;
-                        p.emitted[static_cast<size_t>(b) * (k + 1) + lane] = v;
-                    }
-                    if (k == 32 && lane == 0)
-                        p.emitted[static_cast<size_t>(b) * (k + 1) + 32] = (a == 32 && fix_row >= 0) ? fix_tok : -1;
-                    if (lane == 0) {
-                        p.accept_len[b] = a;
-                        p.n_emitted[b] = a + (fix_row >= 0 ? 1 : 0);
-                    }
-                }
-                if (DISTILL) {
-                    // rows past b_k have no loss: their entries of loss_rows are zero
-                    if (p.loss_rows && lane >= n && lane < k)
-                        p.loss_rows[static_cast<size_t>(b) * k + lane] = 0.f;
-                    float ls = 0.f;
-                    for (int q = 0; q < n; ++q) ls += __shfl_sync(0xffffffffu, r.loss, q);
-                    if (lane == 0) {
-                        p.seq_loss[b] = ls;
-                        p.seq_ticket[b] = 0u;
-                        __threadfence();
-                        const uint32_t old = atomicAdd(&p.hdr->loss_ticket, 1u);
-                        if (old + 1u == static_cast<uint32_t>(p.B)) {
-                            __threadfence();
-                            float tot = 0.f;
-                            for (int s = 0; s < p.B; ++s) tot += __ldcg(p.seq_loss + s);
-                            *p.loss_total = tot;
-                            p.hdr->loss_ticket = 0u;
-                        }
-                    }
-                } else if (lane == 0) {
-                    p.seq_ticket[b] = 0u;
+            } else {
+                const int e_end = min(len, (wv0 + wcnt) * 8);
+                for (int e = wv0 * 8 + lane; e < e_end; e += 32) {
+                    if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + v0 + e] = 0.f;
+                    else static_cast<uint16_t*>(p.dlogits)[drow * V + v0 + e] = 0;
                 }
             }
         }
-        __syncthreads();
-        if (t == 0) { c.kind = c.nkind; c.b = c.nb; c.i = c.ni; }
-        __syncthreads();
-        w = wn;
     }
+    // no CTA leaves while another may still read its shared memory
+    cluster_sync();
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1028,20 +1067,24 @@ __global__ void __launch_bounds__(NT, 1) row_pass_kernel(const RowParams p) {
 namespace {
 
 template <int NT, int NV>
-constexpr size_t smem_bytes() {
-    // staging D, T | delta planes | barriers | control block
-    return ctl_offset<NT, NV>() + sizeof(Ctl<NT / 32>);
+constexpr size_t smem_fixed() {
+    return ctl_offset<NT, NV>() + ((sizeof(Ctl<NT / 32>) + 15) & ~size_t(15));
 }
 
 using KernelFn = void (*)(RowParams);
 
-template <int NT, int NV>
-KernelFn pick_kernel(int flags) {
+template <int NT, int NV, bool AL>
+KernelFn pick_kernel3(int flags) {
     const bool dist = (flags & kFlagDistill) != 0, sto = (flags & kFlagStochastic) != 0;
-    if (dist && sto) return row_pass_kernel<NT, NV, true, true>;
-    if (dist) return row_pass_kernel<NT, NV, true, false>;
-    if (sto) return row_pass_kernel<NT, NV, false, true>;
-    return row_pass_kernel<NT, NV, false, false>;
+    if (dist && sto) return row_pass_kernel<NT, NV, true, true, AL>;
+    if (dist) return row_pass_kernel<NT, NV, true, false, AL>;
+    if (sto) return row_pass_kernel<NT, NV, false, true, AL>;
+    return row_pass_kernel<NT, NV, false, false, AL>;
+}
+
+template <int NT, int NV>
+KernelFn pick_kernel(int flags, bool aligned) {
+    return aligned ? pick_kernel3<NT, NV, true>(flags) : pick_kernel3<NT, NV, false>(flags);
 }
 
 constexpr int kSmallNT = 128, kSmallNV = 2;
@@ -1063,12 +1106,12 @@ bool row_geometry(int V, RowGeometry* g) {
         g->variant = 0;
         g->threads = kSmallNT;
         g->cluster = next_pow2((V + small_cap - 1) / small_cap);
-        g->smem = smem_bytes<kSmallNT, kSmallNV>();
+        g->smem = smem_fixed<kSmallNT, kSmallNV>();
     } else {
         g->variant = 1;
         g->threads = kLargeNT;
         g->cluster = next_pow2((V + large_cap - 1) / large_cap);
-        g->smem = smem_bytes<kLargeNT, kLargeNV>();
+        g->smem = smem_fixed<kLargeNT, kLargeNV>();
     }
     if (g->cluster > 16) return false;
     const int per = (V + g->cluster - 1) / g->cluster;
@@ -1076,33 +1119,44 @@ bool row_geometry(int V, RowGeometry* g) {
     return true;
 }
 
+size_t row_smem_bytes(const RowGeometry& g, int B) {
+    const size_t list = B <= kCompactMaxB ? (static_cast<size_t>(2 * B + 1) * 4 + 15) & ~size_t(15) : 0;
+    return g.smem + list;
+}
+
 int launch_row_pass(const RowParams& p, void* stream) {
     RowGeometry geo;
     if (!row_geometry(p.V, &geo)) return static_cast<int>(cudaErrorInvalidValue);
-    KernelFn fn = geo.variant == 0 ? pick_kernel<kSmallNT, kSmallNV>(p.flags)
-                                   : pick_kernel<kLargeNT, kLargeNV>(p.flags);
+    const bool aligned = p.aligned != 0;
+    KernelFn fn = geo.variant == 0 ? pick_kernel<kSmallNT, kSmallNV>(p.flags, aligned)
+                                   : pick_kernel<kLargeNT, kLargeNV>(p.flags, aligned);
+    const size_t smem = row_smem_bytes(geo, p.B);
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(geo.smem));
+                                           static_cast<int>(smem));
     if (err != cudaSuccess) return static_cast<int>(err);
     if (geo.cluster > 8) {
         err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (err != cudaSuccess) return static_cast<int>(err);
     }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = geo.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (p.pdl) {
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 2;
+    }
     cfg.blockDim = dim3(geo.threads, 1, 1);
-    cfg.dynamicSmemBytes = geo.smem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    // persistent grid: as many clusters as can be resident at once
-    static int cached_clusters[2][17][8] = {};
-    const int fidx = p.flags & 7;
-    int& cache = cached_clusters[geo.variant][geo.cluster][fidx];
+    // persistent grid: as many clusters as can be resident at once (cached per configuration)
+    static int cached_clusters[2][17][8][2] = {};
+    int& cache = cached_clusters[geo.variant][geo.cluster][p.flags & 7][aligned ? 1 : 0];
     if (cache == 0) {
         int dev = 0, sms = 0;
         cudaGetDevice(&dev);
@@ -1110,7 +1164,10 @@ int launch_row_pass(const RowParams& p, void* stream) {
         cfg.gridDim = dim3(geo.cluster * sms, 1, 1);
         int n = 0;
         err = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
-        if (err != cudaSuccess || n < 1) n = sms / geo.cluster > 0 ? sms / geo.cluster : 1;
+        if (err != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = sms / geo.cluster > 0 ? sms / geo.cluster : 1;
+        }
         cache = n;
     }
     const long long max_items = static_cast<long long>(p.B) * (p.kt + p.k);

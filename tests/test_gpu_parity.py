@@ -74,13 +74,15 @@ def compare_sequences(out, D, T, draft, bk_used, seqs, *, mode, tau, seed, step,
             P.assert_close(ri["ratio"][b, :nb], ref["row_ratio"][j, :nb], "ratio seq %d" % b)
         if tie_seq:
             continue
-        if mode == 1 and ref["fix_margin"][j] < P.TIE_SAMPLE:
-            stats["sample_ties"] += 1
-            assert acc_g[j] == ref["accept_len"][j]
-            continue
         assert acc_g[j] == ref["accept_len"][j], (b, acc_g[j], ref["accept_len"][j])
         assert ne_g[j] == ref["n_emitted"][j], b
-        assert np.array_equal(em_g[j], ref["emitted"][j]), (b, em_g[j], ref["emitted"][j])
+        if not np.array_equal(em_g[j], ref["emitted"][j]):
+            # only the sampled correction / bonus token may differ, and only at a near-tie
+            a = int(ref["accept_len"][j])
+            diff = np.nonzero(em_g[j] != ref["emitted"][j])[0]
+            assert mode == 1 and list(diff) == [a] and ref["fix_margin"][j] < P.TIE_SAMPLE, (
+                b, em_g[j], ref["emitted"][j], ref["fix_margin"][j])
+            stats["sample_ties"] += 1
     if check_loss:
         want_grad_for = set(grad_seqs or [])
         sub = [j for j, b in enumerate(seqs) if b in want_grad_for]
@@ -203,7 +205,7 @@ def test_stochastic_qwen_b64_sampled():
     print("stochastic near-ties:", st)
     # the same workload with every b_k = k (full verification)
     out2 = run_fused(w, D, T, draft=draft, use_head=False, bk_in=torch.full((w.B,), w.k, dtype=torch.int32))
-    compare_sequences(out2, D, T, draft, np.full(w.B, w.k, np.int32), seqs[:16], mode=1,
+    compare_sequences(out2, D[:16], T[:16], draft, np.full(w.B, w.k, np.int32), seqs[:16], mode=1,
                       tau=w.tau, seed=w.philox_seed, step=0, lam=w.lam, clip_c=w.clip_c,
                       check_loss=False)
 
@@ -249,5 +251,5 @@ def test_emission_law_v8_million_trials():
         assert abs(ref["row_u"][j, 0] - min(1.0, ref["row_ratio"][j, 0])) < P.TIE_U
     ok = np.ones(n, bool)
     ok[mism] = False
-    ok &= ref["fix_margin"] >= P.TIE_SAMPLE
-    assert np.array_equal(tok[:n][ok], ref["emitted"][ok, 0])
+    differ = ok & (tok[:n] != ref["emitted"][:, 0])
+    assert (ref["fix_margin"][differ] < P.TIE_SAMPLE).all(), np.nonzero(differ)[0][:10]
