@@ -33,7 +33,6 @@ svd_status check_shape(int B, int k, int kt, int V) {
 
 struct WsPtrs {
     WsHeader* hdr;
-    uint32_t* seq_ticket;
     svd_row_info* rec;
     float* seq_loss;
     float* zpart;
@@ -46,7 +45,6 @@ WsPtrs carve(void* ws, int B, int k, int kt, int M) {
     char* base = static_cast<char*>(ws);
     WsPtrs w;
     w.hdr = reinterpret_cast<WsHeader*>(base);
-    w.seq_ticket = reinterpret_cast<uint32_t*>(base + L.seq_ticket);
     w.rec = reinterpret_cast<svd_row_info*>(base + L.rec);
     w.seq_loss = reinterpret_cast<float*>(base + L.seq_loss);
     w.zpart = reinterpret_cast<float*>(base + L.zpart);
@@ -97,7 +95,7 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
     p.dlogits = dlogits; p.loss_rows = loss_rows; p.loss_total = loss_total;
     p.accept_len = accept_len; p.emitted = emitted; p.n_emitted = n_emitted;
     p.row_info = row_info;
-    p.hdr = w.hdr; p.seq_ticket = w.seq_ticket; p.rec = w.rec; p.seq_loss = w.seq_loss;
+    p.hdr = w.hdr; p.rec = w.rec; p.seq_loss = w.seq_loss;
     p.wait_limit_ns = kWaitLimitNs;
     p.pdl = pdl;
     return from_cuda(launch_row_pass(p, stream));

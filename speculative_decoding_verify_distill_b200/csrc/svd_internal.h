@@ -16,7 +16,7 @@ namespace svd {
 struct WsHeader {
     uint32_t status;       // first device-side error (svd_status), sticky until read
     uint32_t head_ticket;  // length head: CTAs finished
-    uint32_t loss_ticket;  // row pass: sequences finished
+    uint32_t loss_ticket;  // finalize pass: CTAs finished
     uint32_t pad[61];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte line");
@@ -35,15 +35,13 @@ __host__ __device__ inline int head_nsplit(int B, int M) {
 }
 
 struct WsLayout {
-    size_t seq_ticket, rec, seq_loss, zpart, part, tile_ticket, total;
+    size_t rec, seq_loss, zpart, part, tile_ticket, total;
 };
 
 __host__ __device__ inline WsLayout ws_layout(int B, int k, int kt, int M) {
     (void)k;
     WsLayout L;
     size_t off = sizeof(WsHeader);
-    L.seq_ticket = off;
-    off = align256(off + sizeof(uint32_t) * (size_t)B);
     L.rec = off;
     off = align256(off + sizeof(svd_row_info) * (size_t)B * (size_t)kt);
     L.seq_loss = off;
@@ -111,7 +109,6 @@ struct RowParams {
     int32_t* n_emitted;
     svd_row_info* row_info;
     WsHeader* hdr;
-    uint32_t* seq_ticket;
     svd_row_info* rec;
     float* seq_loss;
     uint64_t wait_limit_ns;
@@ -125,7 +122,7 @@ int launch_wait_timeout_selftest(WsHeader* hdr, uint64_t limit_ns, void* stream)
 
 // Cluster geometry chosen for a vocabulary size.
 struct RowGeometry {
-    int variant;   // 0: 128 threads x 2 vectors; 1: 512 threads x 5 vectors
+    int variant;   // 0: 128 threads x 2 vectors; 1: 256 x 5; 2: 256 x 10
     int threads;
     int cluster;   // CTAs per row
     int chunk;     // elements per CTA
