@@ -173,6 +173,36 @@ typedef struct svd_verify_distill_args {
 svd_status svd_verify_distill(const svd_verify_distill_args* args, void* ws, size_t ws_bytes,
                               void* stream);
 
+/* Largest workspace svd_verify_distill_noalloc can stand in for (4 MiB per device). */
+#define SVD_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+/* svd_verify_distill without a caller workspace, for callers that cannot allocate device
+ * memory: a C host program with no device allocator, or a runtime that has claimed nearly all
+ * HBM for its own pools and forbids cudaMalloc on its path (cudaMalloc may synchronise the
+ * device and fails once the memory is claimed).  The paper has no counterpart: it is a
+ * deployment variant of the fused call above, with identical arguments, kernels and results.
+ *
+ * Scratch: a file-scope device array of SVD_NOALLOC_SCRATCH_BYTES in the library, one per
+ * device.  Nothing is allocated, by the library or by anything it calls.
+ *   - Set-up: the first call on each device (with that device current; `stream` must belong
+ *     to the current device) looks up the array's address and caches it.  Make that first
+ *     call before any stream capture begins.
+ *   - Zeroing: every call clears the svd_workspace_bytes(B, k, kt, M) bytes it uses with one
+ *     cudaMemsetAsync on `stream`, so nothing needs to start at zero and an earlier device
+ *     error leaves nothing behind.
+ *   - Size limit: calls whose svd_workspace_bytes(B, k, kt, M) exceeds
+ *     SVD_NOALLOC_SCRATCH_BYTES return SVD_ERR_WORKSPACE before anything is launched.
+ *   - Concurrency: all calls on one device share the one array.  Calls that overlap on the
+ *     GPU (different streams, or host threads enqueuing without ordering) race on it and give
+ *     undefined results; order them on one stream or with events.
+ *   - Device errors: if `status_out` (a caller-owned DEVICE pointer to one uint32_t) is not
+ *     NULL, the call's device status word (SVD_OK, SVD_ERR_TOKEN_RANGE or SVD_ERR_TIMEOUT) is
+ *     copied there on `stream` after the kernels.
+ * Other return codes as for svd_verify_distill; SVD_ERR_UNSUPPORTED for a device ordinal
+ * of 64 or more. */
+svd_status svd_verify_distill_noalloc(const svd_verify_distill_args* args, uint32_t* status_out,
+                                      void* stream);
+
 /* Reads and clears the device status word of `ws` (synchronizes `stream`).  Returns SVD_OK,
  * SVD_ERR_TOKEN_RANGE or SVD_ERR_TIMEOUT as recorded by kernels that used this workspace, or
  * SVD_ERR_CUDA if the read itself failed. */

@@ -79,8 +79,10 @@ def lib():
     L.svd_status_string.argtypes = [_I]
     L.svd_status_string.restype = ctypes.c_char_p
     L.svd_selftest_wait_timeout.argtypes = [_P, _SZ, _U64, _P]
+    L.svd_verify_distill_noalloc.argtypes = [ctypes.POINTER(VerifyDistillArgs), _P, _P]
     for fn in ("svd_workspace_reset", "svd_length_head", "svd_verify", "svd_distill_loss_grad",
-               "svd_verify_distill", "svd_get_device_error", "svd_selftest_wait_timeout"):
+               "svd_verify_distill", "svd_get_device_error", "svd_selftest_wait_timeout",
+               "svd_verify_distill_noalloc"):
         getattr(L, fn).restype = _I
     _lib = L
     return L
@@ -283,6 +285,22 @@ class VerifyDistill:
 def svd_verify_distill(D, T, **kw) -> dict:
     """a1-a5 in one call; keyword arguments as in :class:`VerifyDistill`."""
     return VerifyDistill(D, T, **kw)().outputs()
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def svd_verify_distill_noalloc(vd: VerifyDistill, status_out=None, stream=None) -> None:
+    """The fused call on the library's static per-device scratch instead of ``vd.ws``.
+
+    For callers that cannot allocate device memory on their path (a runtime that has claimed
+    nearly all HBM for its own pools, or a host program without a device allocator): the C
+    entry point allocates nothing.  ``status_out`` is an optional one-element int32/uint32 CUDA
+    tensor that receives the device status word.  Overlapping calls on one device race on the
+    shared scratch; the first call per device must come before any stream capture.
+    """
+    _check(lib().svd_verify_distill_noalloc(ctypes.byref(vd.args), _ptr(status_out),
+                                            _stream(stream)), "svd_verify_distill_noalloc")
 
 
 def svd_selftest_wait_timeout(ws: Workspace, limit_ns: int, stream=None) -> None:
