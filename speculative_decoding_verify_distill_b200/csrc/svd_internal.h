@@ -17,7 +17,9 @@ struct WsHeader {
     uint32_t status;       // first device-side error (svd_status), sticky until read
     uint32_t head_ticket;  // length head: CTAs finished
     uint32_t loss_ticket;  // finalize pass: CTAs finished
-    uint32_t pad[61];
+    uint32_t item_ticket;  // row pass: next loaded row to hand out (reset by the finalize pass)
+    uint32_t zero_ticket;  // row pass: next zero-gradient unit to hand out (reset likewise)
+    uint32_t pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte line");
 

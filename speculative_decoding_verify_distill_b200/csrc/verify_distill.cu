@@ -15,8 +15,10 @@
 //     vocabulary, several CTAs per SM).  A cluster owns one logit row at a time; each CTA a
 //     contiguous slice of the vocabulary; each warp a contiguous run of 16-byte vectors of the
 //     slice.  Loaded work items (verified rows and bonus rows) form a compact list (prefix sums
-//     of loaded rows per sequence); cluster c takes items c, c + #clusters, ...  Zero-only
-//     gradient rows follow in a second phase without cluster barriers.
+//     of loaded rows per sequence) handed out one row at a time from a workspace ticket, so a
+//     cluster that starts late (behind the length head, or beside other work) simply takes fewer
+//     rows.  Zero-only gradient rows follow, in quarter-row units handed out to single CTAs,
+//     without cluster barriers.
 //   * Each warp stages its run of D and T in shared memory with its own 1-D bulk copies
 //     (cp.async.bulk, no multicast) on its own mbarrier.  The staged bf16 slice is the only copy:
 //     every pass re-reads it, so a CTA holds no per-element state in registers and several CTAs
@@ -84,11 +86,17 @@ struct Ctl {
     Deposit dep[2];
     Pending pend;
     int wscan[NW];             // prologue scan of the loaded-row counts
+    int wscanz[NW];            // ... and of the zero-gradient row counts
+    int next_w[2];             // rank 0: the next loaded item, by row parity (read over DSMEM)
+    int zs;                    // zero phase: the CTA's next unit
 };
 
-// Batches up to this size keep b_k and the prefix of loaded rows per sequence in shared memory
-// (compact item list); larger batches walk the uncompacted (sequence, row) slots.
+// Batches up to this size keep b_k and the prefixes of loaded and zero-gradient rows per sequence
+// in shared memory (compact lists, handed out dynamically); larger batches walk the uncompacted
+// (sequence, row) slots in a fixed order.
 constexpr int kCompactMaxB = 4096;
+// Zero-gradient rows are handed out in quarters (about 75 KB of stores each at V = 151936).
+constexpr int kZeroSplit = 4;
 
 struct Item {
     int kind, b, i;
@@ -111,6 +119,11 @@ __device__ __forceinline__ int loaded_rows(int n, int kt, bool verify) {
 __device__ __forceinline__ bool zero_row_pred(int k, int n, int i, bool verify) {
     return i < k && (verify ? (n < i) : (n <= i));
 }
+// How many there are in a sequence, and the first of them.
+__device__ __forceinline__ int zero_rows(int k, int n, bool verify) {
+    return verify ? max(0, k - n - 1) : k - n;
+}
+__device__ __forceinline__ int first_zero_row(int n, bool verify) { return verify ? n + 1 : n; }
 
 // b_k of sequence b: from shared memory (compact mode) or global memory (clamped).
 struct BkView {
@@ -262,9 +275,11 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     uint4* stageT = stageD + NV * NT;
     uint64_t* full = reinterpret_cast<uint64_t*>(stageT + NV * NT);
     Ctl<NW>& c = *reinterpret_cast<Ctl<NW>*>(smem_raw + ctl_offset<NT, NV>());
-    // compact mode: b_k [B] and the prefix of loaded rows [B + 1] follow the control block
+    // compact mode: b_k [B] and the prefixes of loaded and zero rows [B + 1] each follow the
+    // control block
     int* sbk = reinterpret_cast<int*>(smem_raw + ctl_offset<NT, NV>() + ((sizeof(Ctl<NW>) + 15) & ~size_t(15)));
     int* spre = sbk + p.B;
+    int* zpre = spre + p.B + 1;
 
     // the finalize pass may be scheduled as soon as SM resources allow; it waits for this grid
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -315,34 +330,46 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     const bool compact = p.B <= kCompactMaxB;
     if (compact) {
         // b_k and the exclusive prefix of loaded rows per sequence, in shared memory
-        int carry = 0;
+        int carry = 0, carryz = 0;
         for (int c0 = 0; c0 < p.B; c0 += NT) {
             const int b = c0 + t;
-            int n = 0, L = 0;
+            int n = 0, L = 0, Z = 0;
             if (b < p.B) {
                 n = clamp_bk(p, __ldg(p.bk + b));
                 L = loaded_rows(n, kt, verify);
+                Z = DISTILL ? zero_rows(k, n, verify) : 0;
                 sbk[b] = n;
             }
-            int incl = L;
+            int incl = L, inclz = Z;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
+                const int yz = __shfl_up_sync(0xffffffffu, inclz, o);
+                if (lane >= o) { incl += y; inclz += yz; }
             }
-            if (lane == 31) c.wscan[warp] = incl;
+            if (lane == 31) { c.wscan[warp] = incl; c.wscanz[warp] = inclz; }
             __syncthreads();
-            int before = 0, tot = 0;
+            int before = 0, tot = 0, beforez = 0, totz = 0;
             for (int q = 0; q < NW; ++q) {
-                const int v = c.wscan[q];
-                if (q < warp) before += v;
+                const int v = c.wscan[q], vz = c.wscanz[q];
+                if (q < warp) { before += v; beforez += vz; }
                 tot += v;
+                totz += vz;
             }
-            if (b < p.B) spre[b] = carry + before + incl - L;
+            if (b < p.B) {
+                spre[b] = carry + before + incl - L;
+                zpre[b] = carryz + beforez + inclz - Z;
+            }
             carry += tot;
+            carryz += totz;
             __syncthreads();
         }
-        if (t == 0) spre[p.B] = carry;
+        if (t == 0) {
+            spre[p.B] = carry;
+            zpre[p.B] = carryz;
+            // the cluster's first loaded item
+            if (rank == 0) c.next_w[0] = static_cast<int>(atomicAdd(&p.hdr->item_ticket, 1u));
+        }
     }
     __syncthreads();
     cluster_sync();  // barriers, deposit slots and the item list ready everywhere
@@ -350,7 +377,15 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     const BkView bkv{compact ? sbk : nullptr, p.bk};
     const int* list = compact ? spre : nullptr;
     const int nslots = loaded_slots(p, list);
-    // the cluster's loaded items are slots cid, cid + ncl, ...; holes are skipped
+    // Compact mode: rank 0 takes the cluster's loaded items one at a time from the workspace
+    // ticket, one row ahead, and every warp reads the index from rank 0 over DSMEM (slot by row
+    // parity: written before barrier #1 of one row, read after it, rewritten two rows later).
+    // Otherwise the cluster's items are slots cid, cid + ncl, ...; holes are skipped.
+    auto shared_item = [&](int slot) -> int {
+        int wv = 0;
+        if (lane == 0) wv = static_cast<int>(dsmem_ld_u32(dsmem_map(&c.next_w[slot], 0)));
+        return __shfl_sync(0xffffffffu, wv, 0);
+    };
     auto next_loaded = [&](int& w) -> Item {
         while (w < nslots) {
             const Item it = decode_loaded(p, list, bkv, w, verify);
@@ -372,9 +407,10 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         }
     };
 
-    int w = cid;
-    Item cur = next_loaded(w);
+    int w = compact ? shared_item(0) : cid;
+    Item cur = compact ? decode_loaded(p, list, bkv, w, verify) : next_loaded(w);
     if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
+    int iter = 0;                // loaded rows done by this cluster (parity of next_w)
     uint32_t phase = 0;          // parity of this warp's staging barrier
     bool wait_dead = false;      // a bounded wait ran out: skip later waits so the kernel ends
     int par = 0;                 // parity of the loaded rows (deposit double buffer)
@@ -414,7 +450,11 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     // ---------------------------------------------------------------- loaded rows
     while (cur.kind != kItemNone) {
         int wn = w + ncl;
-        const Item nxt = next_loaded(wn);
+        Item nxt{kItemNone, -1, -1};
+        if (!compact) nxt = next_loaded(wn);
+        // rank 0 asks for the next item now; the answer is stored before barrier #1
+        int fetched = 0;
+        if (compact && rank == 0 && t == 0) fetched = static_cast<int>(atomicAdd(&p.hdr->item_ticket, 1u));
         const int b = cur.b, i = cur.i;
         const size_t drow = static_cast<size_t>(b) * k + i;      // draft / gradient row
         const size_t trow = static_cast<size_t>(b) * kt + i;     // target row
@@ -558,7 +598,12 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             const Part1 r = warp_reduce_part1(a, k2);
             if (lane == 0) c.cta1 = r;
         }
+        if (compact && rank == 0 && t == 0) c.next_w[(iter + 1) & 1] = fetched;
         cluster_sync();  // #1
+        if (compact) {
+            wn = shared_item((iter + 1) & 1);
+            nxt = decode_loaded(p, list, bkv, wn, verify);
+        }
 
         // ------------------------------------------------ row statistics (every warp)
         float MD, MT, lseD = kQNaN, lseT = kQNaN, L2D = 0.f, L2T = 0.f, dl = 0.f, rkl = 0.f, smax = 0.f;
@@ -920,6 +965,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         par ^= 1;
         cur = nxt;
         w = wn;
+        ++iter;
     }
     if (pending) {  // uniform: every rank walked the same items
         cluster_sync();
@@ -927,7 +973,48 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     }
 
     // ---------------------------------------------------------------- zero-only gradient rows
-    if (DISTILL) {
+    if (DISTILL && compact) {
+        // quarters of the zero rows in the compact list, handed to CTAs one at a time (the next
+        // unit is requested while the current one is written)
+        const int units = zpre[p.B] * kZeroSplit;
+        if (t == 0) c.zs = static_cast<int>(atomicAdd(&p.hdr->zero_ticket, 1u));
+        __syncthreads();
+        int u = c.zs;
+        __syncthreads();
+        while (u < units) {
+            int nextu = 0;
+            if (t == 0) nextu = static_cast<int>(atomicAdd(&p.hdr->zero_ticket, 1u));
+            const int j = u / kZeroSplit, qq = u % kZeroSplit;
+            int lo = 0, hi = p.B;  // largest b with zpre[b] <= j
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (zpre[mid] <= j) lo = mid; else hi = mid;
+            }
+            const int i = first_zero_row(sbk[lo], verify) + (j - zpre[lo]);
+            const size_t drow = static_cast<size_t>(lo) * k + i;
+            if (ALIGNED) {
+                const uint4 zz = make_uint4(0, 0, 0, 0);
+                const int per_elem = p.dl_fp32 ? 2 : 1;       // 16-byte stores per 8 ids
+                const int nv = (V / 8) * per_elem;
+                const int a0 = static_cast<int>(static_cast<long long>(nv) * qq / kZeroSplit);
+                const int a1 = static_cast<int>(static_cast<long long>(nv) * (qq + 1) / kZeroSplit);
+                uint4* g = p.dl_fp32 ? reinterpret_cast<uint4*>(static_cast<float*>(p.dlogits) + drow * V)
+                                     : reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dlogits) + drow * V);
+                for (int e = a0 + t; e < a1; e += NT) __stcs(g + e, zz);
+            } else {
+                const int a0 = static_cast<int>(static_cast<long long>(V) * qq / kZeroSplit);
+                const int a1 = static_cast<int>(static_cast<long long>(V) * (qq + 1) / kZeroSplit);
+                for (int e = a0 + t; e < a1; e += NT) {
+                    if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + e] = 0.f;
+                    else static_cast<uint16_t*>(p.dlogits)[drow * V + e] = 0;
+                }
+            }
+            if (t == 0) c.zs = nextu;
+            __syncthreads();
+            u = c.zs;
+            __syncthreads();
+        }
+    } else if (DISTILL) {
         for (int z = cid; z < p.B * k; z += ncl) {
             const int b = z / k, i = z % k;
             if (!zero_row_pred(k, bkv(p, b), i, verify)) continue;
@@ -962,6 +1049,11 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
 __global__ void __launch_bounds__(256) finalize_kernel(const RowParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ int last;
+    // the row pass has finished: its work tickets go back to zero for the next call
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        p.hdr->item_ticket = 0u;
+        p.hdr->zero_ticket = 0u;
+    }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool verify = (p.flags & kFlagVerify) != 0;
     const bool distill = (p.flags & kFlagDistill) != 0;
@@ -1100,7 +1192,8 @@ bool row_geometry(int V, RowGeometry* g) {
 }
 
 size_t row_smem_bytes(const RowGeometry& g, int B) {
-    const size_t list = B <= kCompactMaxB ? (static_cast<size_t>(2 * B + 1) * 4 + 15) & ~size_t(15) : 0;
+    // compact mode: b_k [B], loaded-row prefix [B + 1], zero-row prefix [B + 1]
+    const size_t list = B <= kCompactMaxB ? (static_cast<size_t>(3 * B + 2) * 4 + 15) & ~size_t(15) : 0;
     return g.smem + list;
 }
 
