@@ -51,23 +51,26 @@ constexpr uint32_t kNone = 0xffffffffu;
 
 enum ItemKind : int { kItemNone = 0, kItemRow = 1, kItemBonus = 2 };
 
-// Per-warp / per-CTA partials of the two cluster reductions.  Sums are relative to the maxima
-// they travel with (exp(x - m) in the log2-scaled domain).
-struct alignas(16) Part1 {
-    float mD, sD, sDd, dmax;   // max D, sum exp, sum exp * (D - T), max (D - T)
-    float mT, sT, pad0, pad1;  // max T, sum exp
+// Messages of the per-row exchanges.  Every CTA of a cluster sends its message to every CTA
+// (itself included) with st.async into the receiver's shared memory; the bytes complete the
+// receiver's exchange barrier, so a CTA waits only for the data it needs and no cluster-wide
+// barrier (with its release fence over the CTA's outstanding gradient stores) is taken per row.
+// Sums travel relative to the maxima they come with (2^((x - m) k2), k2 = log2(e) / tau).
+struct alignas(16) Msg1 {          // after pass A
+    float mD, sD, sDd, dmax;        // max D, sum 2^((D - mD) k2), sum of those times (D - T), max (D - T)
+    float mT, sT;                   // max T, sum 2^((T - mT) k2)
+    uint32_t argT, argD;            // lowest id holding mT / mD in the sender's slice
+    uint32_t prev_tok;              // token the sender sampled for the previous row, or none
+    float prev_ce;                  // -log q_y of the previous row from the owner of y, else 0
+    uint32_t next_item;             // rank 0: the cluster's next loaded item (packed)
+    uint32_t pad;
 };
-struct alignas(16) Part2 {
+struct alignas(16) Msg2 {          // after pass B
     float clip_d, clip_q, n_clip, pad0;    // clipped reverse-KL entries
     unsigned long long mass;               // sample mass (2^-48 units)
     unsigned long long pad1;
 };
-// Deposit targets in rank 0, double-buffered by row parity (read one row later).
-struct alignas(16) Deposit {
-    uint32_t argD, argT;       // lowest index holding the row max (red.min)
-    uint32_t tok;              // sampled token (red.min)
-    float ce;                  // -log q_y, from the owner of y
-};
+static_assert(sizeof(Msg1) == 48 && sizeof(Msg2) == 32, "message sizes are multiples of 16 bytes");
 // Row values rank 0 keeps until the record is written.
 struct Pending {
     int b, i, kind;
@@ -77,18 +80,19 @@ struct Pending {
 
 template <int NW>
 struct Ctl {
-    Part1 p1[NW];              // per-warp partials (local)
-    Part2 p2[NW];
-    Part1 cta1;                // CTA partials, read by every warp of the cluster over DSMEM
-    Part2 cta2;
-    Part2 cta3;                // fallback reduction (residual mass zero: sample from p)
-    unsigned long long wpre[NW];  // exclusive prefix of the warps' sample masses in this CTA
-    Deposit dep[2];
+    Msg1 w1[NW];                    // per-warp partials (local)
+    Msg2 w2[NW];
+    Msg1 in1[2][16];                // exchange #1 by row parity and sender rank
+    Msg2 in2[16];                   // exchange #2 by sender rank
+    unsigned long long in3[16];     // fallback exchange (residual mass zero: sample from p)
+    uint64_t x1[2], x2, x3;         // exchange barriers
+    uint32_t my_tok[2];             // token sampled in this CTA, by row parity
+    float my_ce[2];                 // -log q_y computed in this CTA, by row parity
     Pending pend;
-    int wscan[NW];             // prologue scan of the loaded-row counts
-    int wscanz[NW];            // ... and of the zero-gradient row counts
-    int next_w[2];             // rank 0: the next loaded item, by row parity (read over DSMEM)
-    int zs;                    // zero phase: the CTA's next unit
+    int wscan[NW];                  // prologue scan of the loaded-row counts
+    int wscanz[NW];                 // ... and of the zero-gradient row counts
+    uint32_t first_item;            // rank 0: the cluster's first loaded item (packed)
+    int zs;                         // zero phase: the CTA's next unit
 };
 
 // Batches up to this size keep b_k and the prefixes of loaded and zero-gradient rows per sequence
@@ -101,6 +105,43 @@ constexpr int kZeroSplit = 4;
 struct Item {
     int kind, b, i;
 };
+// Items travel between CTAs as one word: (b << 8) | (i << 2) | kind; 0 means none.
+__device__ __forceinline__ uint32_t pack_item(const Item& it) {
+    return it.kind == kItemNone ? 0u
+                                : (static_cast<uint32_t>(it.b) << 8) | (static_cast<uint32_t>(it.i) << 2) |
+                                      static_cast<uint32_t>(it.kind);
+}
+__device__ __forceinline__ Item unpack_item(uint32_t v) {
+    if ((v & 3u) == 0u) return Item{kItemNone, -1, -1};
+    return Item{static_cast<int>(v & 3u), static_cast<int>(v >> 8), static_cast<int>((v >> 2) & 63u)};
+}
+// Position (0..7) of the first element of a bf16 vector equal to R (7 if none: never used then).
+__device__ __forceinline__ int first_pos(const uint4& v, float R) {
+    float x[8];
+    unpack8(v, x);
+    int l = 7;
+#pragma unroll
+    for (int q = 6; q >= 0; --q) l = (x[q] == R) ? q : l;
+    return l;
+}
+// The four bf16 pairs of a 16-byte vector as packed fp32 pairs (exact).
+__device__ __forceinline__ void unpack8x2(const uint4& v, float2 (&x)[4]) {
+    x[0] = make_float2(bf_lo(v.x), bf_hi(v.x));
+    x[1] = make_float2(bf_lo(v.y), bf_hi(v.y));
+    x[2] = make_float2(bf_lo(v.z), bf_hi(v.z));
+    x[3] = make_float2(bf_lo(v.w), bf_hi(v.w));
+}
+__device__ __forceinline__ Msg1 empty_msg1() {
+    Msg1 m;
+    m.mD = m.mT = m.dmax = kNegInf;
+    m.sD = m.sDd = m.sT = 0.f;
+    m.argT = m.argD = kNone;
+    m.prev_tok = kNone;
+    m.prev_ce = 0.f;
+    m.next_item = 0u;
+    m.pad = 0u;
+    return m;
+}
 
 __device__ __forceinline__ int clamp_bk(const RowParams& p, int n) {
     if (n < 1 || n > p.k) {
@@ -165,11 +206,6 @@ __device__ __forceinline__ int loaded_slots(const RowParams& p, const int* spre)
     return spre ? spre[p.B] : p.B * p.kt;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -180,36 +216,10 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
-// Scale factor that moves a sum relative to max m onto the common max M (0 for empty sums).
+// Factor that moves a sum taken relative to reference round(m k2) onto round(M k2) (exactly 1
+// when m == M).  Maxima at or below -1e38 mark empty sums (all -inf, or the staging sentinel).
 __device__ __forceinline__ float rescale(float m, float M, float k2) {
-    return m == kNegInf ? 0.f : fast_exp2((m - M) * k2);
-}
-// Reduces per-lane Part1 values over the warp: maxima first, then one rescale per lane, then
-// plain sums; every lane ends with the result.
-__device__ __forceinline__ Part1 warp_reduce_part1(const Part1& a, float k2) {
-    Part1 r;
-    r.mD = warp_max(a.mD);
-    r.mT = warp_max(a.mT);
-    r.dmax = warp_max(a.dmax);
-    const float cD = rescale(a.mD, r.mD, k2), cT = rescale(a.mT, r.mT, k2);
-    r.sD = warp_sum(a.sD * cD);
-    r.sDd = warp_sum(a.sDd * cD);
-    r.sT = warp_sum(a.sT * cT);
-    r.pad0 = r.pad1 = 0.f;
-    return r;
-}
-__device__ __forceinline__ Part1 empty_part1() {
-    Part1 r;
-    r.mD = r.mT = r.dmax = kNegInf;
-    r.sD = r.sDd = r.sT = 0.f;
-    r.pad0 = r.pad1 = 0.f;
-    return r;
-}
-__device__ __forceinline__ float sum8(const float (&v)[8]) {
-    return ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
-}
-__device__ __forceinline__ float max8f(const float (&v)[8]) {
-    return fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
+    return m > -1e38f ? fast_exp2(__fsub_rn(__fmul_rn(m, k2), __fmul_rn(M, k2))) : 0.f;
 }
 
 // Per-element quantities with explicit rounding (no contraction), so that the values summed in
@@ -237,17 +247,6 @@ __device__ __forceinline__ unsigned long long scale_mass(unsigned long long R, u
     return (lo >> 24) | (hi << 40);
 }
 
-__device__ __forceinline__ void dsmem_ld4(uint32_t a, float (&v)[4]) {
-    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
-                 : "r"(a)
-                 : "memory");
-}
-__device__ __forceinline__ unsigned long long dsmem_ld_u64(uint32_t a) {
-    unsigned long long v;
-    asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
-    return v;
-}
 
 __device__ __forceinline__ void warp_inclusive_scan_u64(unsigned long long& x) {
     const int lane = threadIdx.x & 31;
@@ -290,6 +289,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     const int cid = static_cast<int>(cluster_id_x());
     const int ncl = static_cast<int>(num_clusters_x());
     const bool verify = (p.flags & kFlagVerify) != 0;
+    const bool greedy_x = verify && p.draft == nullptr;   // draft token = argmax of the draft row
     const int V = p.V, k = p.k, kt = p.kt;
     const int v0 = static_cast<int>(rank) * p.chunk;
     const int len = max(0, min(p.chunk, V - v0));
@@ -298,20 +298,21 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     const int vpw = (nvec + NW - 1) / NW;
     const int wv0 = min(nvec, warp * vpw);
     const int wcnt = max(0, min(nvec, wv0 + vpw) - wv0);
-    const float k2 = p.k2, itau = p.inv_tau;
+    const float k2 = p.k2, itau = p.inv_tau, cc = p.clip_c;
     uint4* myD = stageD + warp * NV * 32;
     uint4* myT = stageT + warp * NV * 32;
 
     // ---------------------------------------------------------------- prologue
     if (t == 0) {
         for (int q = 0; q < NW; ++q) mbar_init(&full[q], 1);
+        mbar_init(&c.x1[0], 1);
+        mbar_init(&c.x1[1], 1);
+        mbar_init(&c.x2, 1);
+        mbar_init(&c.x3, 1);
         fence_mbar_init();
-        for (int q = 0; q < 2; ++q) {
-            c.dep[q].argD = kNone;
-            c.dep[q].argT = kNone;
-            c.dep[q].tok = kNone;
-            c.dep[q].ce = 0.f;
-        }
+        c.my_tok[0] = c.my_tok[1] = kNone;
+        c.my_ce[0] = c.my_ce[1] = 0.f;
+        c.first_item = 0u;
     }
     // Vectors past the end of a warp's run hold a finite sentinel (the most negative bf16) in
     // both D and T: its exp is 0 and D - T is 0, so the passes run straight-line code over all
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const bool compact = p.B <= kCompactMaxB;
     if (compact) {
-        // b_k and the exclusive prefix of loaded rows per sequence, in shared memory
+        // b_k and the exclusive prefixes of loaded rows and zero-gradient rows per sequence
         int carry = 0, carryz = 0;
         for (int c0 = 0; c0 < p.B; c0 += NT) {
             const int b = c0 + t;
@@ -367,25 +368,22 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         if (t == 0) {
             spre[p.B] = carry;
             zpre[p.B] = carryz;
-            // the cluster's first loaded item
-            if (rank == 0) c.next_w[0] = static_cast<int>(atomicAdd(&p.hdr->item_ticket, 1u));
+            // rank 0 takes the cluster's first loaded item from the workspace ticket
+            if (rank == 0) {
+                const int w0 = static_cast<int>(atomicAdd(&p.hdr->item_ticket, 1u));
+                c.first_item = pack_item(decode_loaded(p, spre, BkView{sbk, p.bk}, w0, verify));
+            }
         }
     }
     __syncthreads();
-    cluster_sync();  // barriers, deposit slots and the item list ready everywhere
+    cluster_sync();  // barriers, lists and the first item ready everywhere
 
     const BkView bkv{compact ? sbk : nullptr, p.bk};
     const int* list = compact ? spre : nullptr;
     const int nslots = loaded_slots(p, list);
-    // Compact mode: rank 0 takes the cluster's loaded items one at a time from the workspace
-    // ticket, one row ahead, and every warp reads the index from rank 0 over DSMEM (slot by row
-    // parity: written before barrier #1 of one row, read after it, rewritten two rows later).
-    // Otherwise the cluster's items are slots cid, cid + ncl, ...; holes are skipped.
-    auto shared_item = [&](int slot) -> int {
-        int wv = 0;
-        if (lane == 0) wv = static_cast<int>(dsmem_ld_u32(dsmem_map(&c.next_w[slot], 0)));
-        return __shfl_sync(0xffffffffu, wv, 0);
-    };
+    // Compact mode: rank 0 takes loaded items one at a time from the workspace ticket, one row
+    // ahead, and passes each in its exchange message.  Otherwise the cluster's items are slots
+    // cid, cid + ncl, ...; holes are skipped.
     auto next_loaded = [&](int& w) -> Item {
         while (w < nslots) {
             const Item it = decode_loaded(p, list, bkv, w, verify);
@@ -407,54 +405,105 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         }
     };
 
-    int w = compact ? shared_item(0) : cid;
-    Item cur = compact ? decode_loaded(p, list, bkv, w, verify) : next_loaded(w);
+    // gradient stores of one 8-id vector (lv: index in this warp's run) of row drow
+    auto store_vec = [&](size_t drow, int lv, const float2 (&g)[4]) {
+        const int base = v0 + (wv0 + lv) * 8;
+        if (ALIGNED) {
+            if (p.dl_fp32) {
+                float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.dlogits) + drow * V + base);
+                __stcs(o, make_float4(g[0].x, g[0].y, g[1].x, g[1].y));
+                __stcs(o + 1, make_float4(g[2].x, g[2].y, g[3].x, g[3].y));
+            } else {
+                uint4 pk;
+                pk.x = pack_bf16x2(g[0].x, g[0].y);
+                pk.y = pack_bf16x2(g[1].x, g[1].y);
+                pk.z = pack_bf16x2(g[2].x, g[2].y);
+                pk.w = pack_bf16x2(g[3].x, g[3].y);
+                __stcs(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dlogits) + drow * V + base), pk);
+            }
+        } else {
+            const float gl[8] = {g[0].x, g[0].y, g[1].x, g[1].y, g[2].x, g[2].y, g[3].x, g[3].y};
+#pragma unroll
+            for (int l = 0; l < 8; ++l) {
+                if (base + l < V && (wv0 + lv) * 8 + l < len) {
+                    if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + base + l] = gl[l];
+                    else static_cast<uint16_t*>(p.dlogits)[drow * V + base + l] =
+                        static_cast<uint16_t>(pack_bf16x2(gl[l], 0.f) & 0xffffu);
+                }
+            }
+        }
+    };
+    auto store_elem = [&](size_t drow, int id, float g) {
+        if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + id] = g;
+        else static_cast<uint16_t*>(p.dlogits)[drow * V + id] = static_cast<uint16_t>(pack_bf16x2(g, 0.f) & 0xffffu);
+    };
+
+    Item cur{kItemNone, -1, -1};
+    int w = cid;
+    if (compact) {
+        uint32_t v = 0;
+        if (lane == 0) v = dsmem_ld_u32(dsmem_map(&c.first_item, 0));
+        cur = unpack_item(__shfl_sync(0xffffffffu, v, 0));
+    } else {
+        cur = next_loaded(w);
+    }
     if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
-    int iter = 0;                // loaded rows done by this cluster (parity of next_w)
     uint32_t phase = 0;          // parity of this warp's staging barrier
     bool wait_dead = false;      // a bounded wait ran out: skip later waits so the kernel ends
-    int par = 0;                 // parity of the loaded rows (deposit double buffer)
+    int it = 0;                  // loaded rows done (row parity selects the exchange #1 buffers)
+    uint32_t n2 = 0, n3 = 0;     // completed phases of exchange barriers #2 and #3
     bool pending = false;        // rank 0 owes the record of the previous loaded row
 
-    // rank 0, warp NW-1: write the record of the previous loaded row (its deposits are visible)
-    auto write_record = [&]() {
-        if (lane != 0) return;
+    auto wait_x = [&](uint64_t* bar, uint32_t parity) {
+        if (!wait_dead && !mbar_wait_cluster_bounded(bar, parity, p.wait_limit_ns)) {
+            wait_dead = true;
+            set_device_error(&p.hdr->status, SVD_ERR_TIMEOUT);
+        }
+    };
+    // warp 0: message #1 (48 bytes) to every rank of the cluster, lane r -> rank r
+    auto send1 = [&](const uint4& q0, const uint4& q1, const uint4& q2, int par) {
+        if (lane < CL) {
+            const uint32_t dst = dsmem_map(&c.in1[par][rank], static_cast<uint32_t>(lane));
+            const uint32_t bar = dsmem_map(&c.x1[par], static_cast<uint32_t>(lane));
+            st_async_v4(dst, q0, bar);
+            st_async_v4(dst + 16, q1, bar);
+            st_async_v4(dst + 32, q2, bar);
+        }
+    };
+    // rank 0, one lane: the record of the previous loaded row
+    auto write_record = [&](uint32_t tok, float ce) {
         const Pending& pd = c.pend;
-        Deposit& dp = c.dep[par ^ 1];
-        const bool isRow = pd.kind == kItemRow;
         svd_row_info r;
         r.draft_token = pd.x;
         r.target_argmax = pd.y;
         r.accepted = pd.acc;
         if (!verify) r.sample_token = -1;
         else if (!STOCH) r.sample_token = pd.y;
-        else r.sample_token = (pd.do_sample && dp.tok != kNone) ? static_cast<int32_t>(dp.tok) : -1;
+        else r.sample_token = (pd.do_sample && tok != kNone) ? static_cast<int32_t>(tok) : -1;
         r.ratio = pd.ratio;
         r.lse_draft = pd.lseD;
         r.lse_target = pd.lseT;
         float L = 0.f;
-        if (DISTILL && isRow) {
-            L = p.lambda * dp.ce + (1.f - p.lambda) * pd.kc;
+        if (DISTILL && pd.kind == kItemRow) {
+            L = p.lambda * ce + (1.f - p.lambda) * pd.kc;
             if (p.loss_rows) p.loss_rows[static_cast<size_t>(pd.b) * k + pd.i] = L;
         }
         r.loss = L;
         const size_t trow = static_cast<size_t>(pd.b) * kt + pd.i;
         p.rec[trow] = r;
         if (p.row_info) p.row_info[trow] = r;
-        dp.argD = kNone;
-        dp.argT = kNone;
-        dp.tok = kNone;
-        dp.ce = 0.f;
     };
 
     // ---------------------------------------------------------------- loaded rows
     while (cur.kind != kItemNone) {
+        const int par = it & 1;
         int wn = w + ncl;
         Item nxt{kItemNone, -1, -1};
         if (!compact) nxt = next_loaded(wn);
-        // rank 0 asks for the next item now; the answer is stored before barrier #1
-        int fetched = 0;
-        if (compact && rank == 0 && t == 0) fetched = static_cast<int>(atomicAdd(&p.hdr->item_ticket, 1u));
+        // rank 0 asks for the next item now; it travels in this row's message #1
+        uint32_t fetched = 0;
+        if (compact && rank == 0 && t == 0) fetched = atomicAdd(&p.hdr->item_ticket, 1u);
+        if (t == 0) mbar_arrive_expect_tx(&c.x1[par], static_cast<uint32_t>(CL * sizeof(Msg1)));
         const int b = cur.b, i = cur.i;
         const size_t drow = static_cast<size_t>(b) * k + i;      // draft / gradient row
         const size_t trow = static_cast<size_t>(b) * kt + i;     // target row
@@ -531,108 +580,157 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 bjD = upD ? j : bjD;
             }
         }
-        // argmax candidates: the first element equal to the thread maximum in that vector
-        uint32_t candD = kNone, candT = kNone;
+        // argmax candidates: the first id equal to the thread maximum
+        uint32_t candT = kNone, candD = kNone;
         {
-            float xv[8];
-            unpack8(myT[bjT * 32 + lane], xv);
-            int l = 0;
-            while (l < 7 && xv[l] != RT) ++l;
-            candT = static_cast<uint32_t>(v0 + (wv0 + bjT * 32 + lane) * 8 + l);
-        }
-        if (rowVerify && p.draft == nullptr) {
-            float xv[8];
-            unpack8(myD[bjD * 32 + lane], xv);
-            int l = 0;
-            while (l < 7 && xv[l] != RD) ++l;
-            candD = static_cast<uint32_t>(v0 + (wv0 + bjD * 32 + lane) * 8 + l);
+            const int lvT = bjT * 32 + lane;
+            if (lvT < wcnt) candT = static_cast<uint32_t>(v0 + (wv0 + lvT) * 8 + first_pos(myT[lvT], RT));
+            if (greedy_x && isRow) {
+                const int lvD = bjD * 32 + lane;
+                if (lvD < wcnt) candD = static_cast<uint32_t>(v0 + (wv0 + lvD) * 8 + first_pos(myD[lvD], RD));
+            }
         }
         // main pass: exp relative to the thread maxima (no rescaling) and the reverse-KL moment;
         // straight-line over all rounds (sentinel vectors contribute exact zeros).  A thread
         // holding sentinels only keeps a zero reference.
         float emax[NV];
-        float sD = 0.f, sDd = 0.f, sT = 0.f, dmax = kNegInf;
-        const float AD = RD > -1e38f ? RD * k2 : 0.f, AT = RT > -1e38f ? RT * k2 : 0.f;
+        float2 aD = make_float2(0.f, 0.f), aDd = make_float2(0.f, 0.f), aT = make_float2(0.f, 0.f);
+        float dmax = kNegInf;
+        const float AD = RD > -1e38f ? __fmul_rn(RD, k2) : 0.f, AT = RT > -1e38f ? __fmul_rn(RT, k2) : 0.f;
+        const float2 K2 = make_float2(k2, k2);
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
             emax[j] = 0.f;
             if (!need_lse) continue;
             const int lv = j * 32 + lane;
-            float xt[8], et[8];
-            unpack8(myT[lv], xt);
+            float2 xt[4], et[4];
+            unpack8x2(myT[lv], xt);
+            const float2 nAT = make_float2(-AT, -AT);
 #pragma unroll
-            for (int l = 0; l < 8; ++l) et[l] = fast_exp2(fmaf(xt[l], k2, -AT));
-            sT += sum8(et);
+            for (int h = 0; h < 4; ++h) {
+                const float2 a = fma2(xt[h], K2, nAT);
+                et[h] = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+            }
+            aT = add2(aT, add2(add2(et[0], et[1]), add2(et[2], et[3])));
             if (isRow) {
-                float xd[8], ed[8], dd[8];
-                unpack8(myD[lv], xd);
+                float2 xd[4], ed[4];
+                unpack8x2(myD[lv], xd);
+                const float2 nAD = make_float2(-AD, -AD);
 #pragma unroll
-                for (int l = 0; l < 8; ++l) {
-                    ed[l] = fast_exp2(fmaf(xd[l], k2, -AD));
-                    dd[l] = xd[l] - xt[l];
+                for (int h = 0; h < 4; ++h) {
+                    const float2 a = fma2(xd[h], K2, nAD);
+                    ed[h] = make_float2(fast_exp2(a.x), fast_exp2(a.y));
                 }
-                sD += sum8(ed);
-                float a0 = ed[0] * dd[0], a1 = ed[1] * dd[1];
-                a0 = fmaf(ed[2], dd[2], a0); a1 = fmaf(ed[3], dd[3], a1);
-                a0 = fmaf(ed[4], dd[4], a0); a1 = fmaf(ed[5], dd[5], a1);
-                a0 = fmaf(ed[6], dd[6], a0); a1 = fmaf(ed[7], dd[7], a1);
-                sDd += a0 + a1;
+                aD = add2(aD, add2(add2(ed[0], ed[1]), add2(ed[2], ed[3])));
+                float2 dd[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) dd[h] = sub2(xd[h], xt[h]);
+                aDd = fma2(ed[0], dd[0], aDd);
+                aDd = fma2(ed[1], dd[1], aDd);
+                aDd = fma2(ed[2], dd[2], aDd);
+                aDd = fma2(ed[3], dd[3], aDd);
                 if (DISTILL) {
-                    dmax = fmaxf(dmax, max8f(dd));
-                    emax[j] = max8f(ed);
+                    dmax = fmaxf(dmax, fmaxf(fmaxf(fmaxf(dd[0].x, dd[0].y), fmaxf(dd[1].x, dd[1].y)),
+                                             fmaxf(fmaxf(dd[2].x, dd[2].y), fmaxf(dd[3].x, dd[3].y))));
+                    emax[j] = fmaxf(fmaxf(fmaxf(ed[0].x, ed[0].y), fmaxf(ed[1].x, ed[1].y)),
+                                    fmaxf(fmaxf(ed[2].x, ed[2].y), fmaxf(ed[3].x, ed[3].y)));
                 }
             }
         }
 
-        // reduction #1: warp -> CTA (local shared memory) -> cluster (one DSMEM load per rank)
+        // warp partials -> shared memory -> warp 0 -> message #1 to every rank
         {
-            Part1 a;
-            a.mD = RD; a.sD = sD; a.sDd = sDd; a.dmax = dmax; a.mT = RT; a.sT = sT;
-            a.pad0 = a.pad1 = 0.f;
-            const Part1 r = warp_reduce_part1(a, k2);
-            if (lane == 0) c.p1[warp] = r;
+            const float wmD = redux_max_f32(RD), wmT = redux_max_f32(RT);
+            Msg1 m;
+            m.mD = wmD;
+            m.mT = wmT;
+            m.argT = redux_min_u32(RT == wmT ? candT : kNone);
+            m.argD = (greedy_x && isRow) ? redux_min_u32(RD == wmD ? candD : kNone) : kNone;
+            m.sD = m.sDd = m.sT = 0.f;
+            m.dmax = kNegInf;
+            if (need_lse) {
+                m.sT = warp_sum((aT.x + aT.y) * (RT > -1e38f ? fast_exp2(__fsub_rn(AT, __fmul_rn(wmT, k2))) : 0.f));
+                if (isRow) {
+                    const float fD = RD > -1e38f ? fast_exp2(__fsub_rn(AD, __fmul_rn(wmD, k2))) : 0.f;
+                    m.sD = warp_sum((aD.x + aD.y) * fD);
+                    m.sDd = warp_sum((aDd.x + aDd.y) * fD);
+                    if (DISTILL) m.dmax = redux_max_f32(dmax);
+                }
+            }
+            m.prev_tok = kNone;
+            m.prev_ce = 0.f;
+            m.next_item = 0u;
+            m.pad = 0u;
+            if (lane == 0) c.w1[warp] = m;
         }
         __syncthreads();
         if (warp == 0) {
-            const Part1 a = lane < NW ? c.p1[lane] : empty_part1();
-            const Part1 r = warp_reduce_part1(a, k2);
-            if (lane == 0) c.cta1 = r;
+            const Msg1 a = lane < NW ? c.w1[lane] : empty_msg1();
+            const float cmD = redux_max_f32(a.mD), cmT = redux_max_f32(a.mT);
+            const uint32_t cargT = redux_min_u32(a.mT == cmT ? a.argT : kNone);
+            const uint32_t cargD = redux_min_u32(a.mD == cmD ? a.argD : kNone);
+            const float cdmax = redux_max_f32(a.dmax);
+            float csD = 0.f, csDd = 0.f, csT = 0.f;
+            if (need_lse) {
+                const float fT = rescale(a.mT, cmT, k2);
+                csT = warp_sum(a.sT * fT);
+                if (isRow) {
+                    const float fD = rescale(a.mD, cmD, k2);
+                    csD = warp_sum(a.sD * fD);
+                    csDd = warp_sum(a.sDd * fD);
+                }
+            }
+            uint32_t nitem = 0u;
+            if (compact && rank == 0) {
+                const int fw = static_cast<int>(__shfl_sync(0xffffffffu, fetched, 0));
+                nitem = pack_item(decode_loaded(p, list, bkv, fw, verify));
+            }
+            // the previous row's deposits of this CTA go out with this row's message
+            const uint32_t ptok = c.my_tok[par ^ 1];
+            const float pce = c.my_ce[par ^ 1];
+            send1(make_uint4(__float_as_uint(cmD), __float_as_uint(csD), __float_as_uint(csDd), __float_as_uint(cdmax)),
+                  make_uint4(__float_as_uint(cmT), __float_as_uint(csT), cargT, cargD),
+                  make_uint4(ptok, __float_as_uint(pce), nitem, 0u), par);
+            __syncwarp();
+            if (lane == 0) {
+                c.my_tok[par ^ 1] = kNone;
+                c.my_ce[par ^ 1] = 0.f;
+            }
         }
-        if (compact && rank == 0 && t == 0) c.next_w[(iter + 1) & 1] = fetched;
-        cluster_sync();  // #1
-        if (compact) {
-            wn = shared_item((iter + 1) & 1);
-            nxt = decode_loaded(p, list, bkv, wn, verify);
-        }
+        wait_x(&c.x1[par], static_cast<uint32_t>(it >> 1) & 1u);
 
         // ------------------------------------------------ row statistics (every warp)
         float MD, MT, lseD = kQNaN, lseT = kQNaN, L2D = 0.f, L2T = 0.f, dl = 0.f, rkl = 0.f, smax = 0.f;
+        uint32_t y, ptok_all;
         {
-            Part1 a = empty_part1();
-            if (lane < CL) {
-                const uint32_t ad = dsmem_map(&c.cta1, lane);
-                float v[4], u[4];
-                dsmem_ld4(ad, v);
-                dsmem_ld4(ad + 16, u);
-                a.mD = v[0]; a.sD = v[1]; a.sDd = v[2]; a.dmax = v[3]; a.mT = u[0]; a.sT = u[1];
-            }
-            const Part1 r = warp_reduce_part1(a, k2);   // identical in every lane, warp and rank
-            MD = r.mD;
-            MT = r.mT;
+            const Msg1 a = lane < CL ? c.in1[par][lane] : empty_msg1();
+            MD = redux_max_f32(a.mD);
+            MT = redux_max_f32(a.mT);
+            y = redux_min_u32(a.mT == MT ? a.argT : kNone);
+            if (greedy_x && isRow) x = redux_min_u32(a.mD == MD ? a.argD : kNone);
+            ptok_all = redux_min_u32(a.prev_tok);
+            if (compact) nxt = unpack_item(__shfl_sync(0xffffffffu, a.next_item, 0));
             if (need_lse) {
-                if (isRow) lseD = r.mD * itau + logf(r.sD);
-                lseT = r.mT * itau + logf(r.sT);
-                L2D = lseD * kLog2e;
+                const float sT = warp_sum(a.sT * rescale(a.mT, MT, k2));
+                lseT = MT * itau + logf(sT);
                 L2T = lseT * kLog2e;
-                dl = lseD - lseT;
                 if (isRow) {
-                    rkl = (r.sDd / r.sD) * itau - dl;   // sum_v q_v (log q_v - log p_v)
-                    smax = r.dmax * itau - dl;          // largest log q_v - log p_v
+                    const float fD = rescale(a.mD, MD, k2);
+                    const float sD = warp_sum(a.sD * fD);
+                    const float sDd = warp_sum(a.sDd * fD);
+                    lseD = MD * itau + logf(sD);
+                    L2D = lseD * kLog2e;
+                    dl = lseD - lseT;
+                    rkl = (sDd / sD) * itau - dl;   // sum_v q_v (log q_v - log p_v)
+                    if (DISTILL) smax = redux_max_f32(a.dmax) * itau - dl;   // largest log q_v - log p_v
                 }
             }
+            // rank 0 writes the previous row's record (its token and -log q_y arrived just now)
+            if (pending && rank == 0 && warp == NW - 1) {
+                const float pce = warp_sum(a.prev_ce);   // one owner sends it, the rest send 0
+                if (lane == 0) write_record(ptok_all, pce);
+            }
         }
-        // rank 0 writes the previous row's record while the rest of the cluster works
-        if (pending && rank == 0 && warp == NW - 1) write_record();
         pending = false;
 
         // stochastic decision (every warp computes the same value)
@@ -656,21 +754,26 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 do_sample = 1;  // bonus row: sample from p
             }
         }
+        if (rowVerify && !STOCH) acc = (x == y) ? 1 : 0;
 
-        // lazy argmax: only the threads holding the row maximum offer their candidate
-        Deposit* dep0 = &c.dep[par];
-        if (candD != kNone && RD == MD) dsmem_min_u32(dsmem_map(&dep0->argD, 0), candD);
-        if (RT == MT) dsmem_min_u32(dsmem_map(&dep0->argT, 0), candT);
+        // Clipping is possible only if max_v q_v * max_v (log q_v - log p_v) reaches c; the
+        // bound is the same in every CTA, so the second exchange is skipped uniformly.
+        bool do_clip = false;
+        float qthr = 0.f;
+        if (DISTILL && isRow && isfinite(cc) && smax > 0.f) {
+            qthr = (cc / smax) * 0.9999f;
+            const float qmax = fast_exp2(__fsub_rn(__fmul_rn(MD, k2), L2D));
+            do_clip = qmax * 1.001f > qthr;
+        }
+        const bool need_x2 = do_clip || (STOCH && do_sample);
 
         // -------------------------------------------------------- pass B
         // d_v = q_v s_v <= q_v s_max, so only entries with q_v > c / s_max can be clipped; those
         // vectors alone are re-read and tested exactly
         float clip_d = 0.f, clip_q = 0.f, n_clip = 0.f;
         uint32_t clipmask = 0;
-        const float cc = p.clip_c;
-        if (DISTILL && isRow && isfinite(cc) && smax > 0.f) {
+        if (do_clip) {
             const float fD = fast_exp2(AD - L2D);          // q = e * fD for this thread's exps
-            const float qthr = (cc / smax) * 0.9999f;
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
                 if (emax[j] * fD > qthr) {
@@ -713,90 +816,84 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             }
             wmass = warp_sum_u64(wmass);
         }
-        // reduction #2: warp -> CTA (fixed order) -> cluster
-        if (DISTILL && isRow) {
-            clip_d = warp_sum(clip_d);
-            clip_q = warp_sum(clip_q);
-            n_clip = warp_sum(n_clip);
-        }
-        if (lane == 0) {
-            Part2 q2;
-            q2.clip_d = clip_d; q2.clip_q = clip_q; q2.n_clip = n_clip; q2.pad0 = 0.f;
-            q2.mass = wmass;
-            q2.pad1 = 0ull;
-            c.p2[warp] = q2;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-            unsigned long long m = 0ull;
-            if (lane < NW) {
-                const Part2 q = c.p2[lane];
-                a0 = q.clip_d; a1 = q.clip_q; a2 = q.n_clip; m = q.mass;
-            }
+
+        // exchange #2: clip sums and sample masses (skipped when neither is needed)
+        float g_clip_d = 0.f, g_clip_q = 0.f, g_n_clip = 0.f;
+        unsigned long long R = 0ull, before = 0ull;
+        // exclusive prefix of the sample masses of the warps before this one (this CTA)
+        auto warp_prefix = [&](unsigned long long m) -> unsigned long long {
             unsigned long long incl = m;
             warp_inclusive_scan_u64(incl);
-            if (lane < NW) c.wpre[lane] = incl - m;
-            a0 = warp_sum(a0);
-            a1 = warp_sum(a1);
-            a2 = warp_sum(a2);
-            const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
+            return __shfl_sync(0xffffffffu, incl - m, warp);
+        };
+        if (need_x2) {
+            if (t == 0) mbar_arrive_expect_tx(&c.x2, static_cast<uint32_t>(CL * sizeof(Msg2)));
+            if (do_clip) {
+                clip_d = warp_sum(clip_d);
+                clip_q = warp_sum(clip_q);
+                n_clip = warp_sum(n_clip);
+            }
             if (lane == 0) {
-                Part2 q2;
-                q2.clip_d = a0; q2.clip_q = a1; q2.n_clip = a2; q2.pad0 = 0.f;
-                q2.mass = tot;
+                Msg2 q2;
+                q2.clip_d = clip_d; q2.clip_q = clip_q; q2.n_clip = n_clip; q2.pad0 = 0.f;
+                q2.mass = wmass;
                 q2.pad1 = 0ull;
-                c.cta2 = q2;
+                c.w2[warp] = q2;
+            }
+            __syncthreads();
+            const unsigned long long mw = lane < NW ? c.w2[lane].mass : 0ull;
+            unsigned long long wpre = 0ull;
+            if (STOCH && do_sample) wpre = warp_prefix(mw);
+            if (warp == 0) {
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+                if (do_clip && lane < NW) {
+                    a0 = c.w2[lane].clip_d; a1 = c.w2[lane].clip_q; a2 = c.w2[lane].n_clip;
+                }
+                if (do_clip) {
+                    a0 = warp_sum(a0);
+                    a1 = warp_sum(a1);
+                    a2 = warp_sum(a2);
+                }
+                const unsigned long long tot = warp_sum_u64(mw);
+                if (lane < CL) {
+                    const uint32_t dst = dsmem_map(&c.in2[rank], static_cast<uint32_t>(lane));
+                    const uint32_t bar = dsmem_map(&c.x2, static_cast<uint32_t>(lane));
+                    st_async_v4(dst, make_uint4(__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2), 0u), bar);
+                    st_async_v4(dst + 16, make_uint4(static_cast<uint32_t>(tot), static_cast<uint32_t>(tot >> 32), 0u, 0u), bar);
+                }
+            }
+            wait_x(&c.x2, n2 & 1u);
+            ++n2;
+            const Msg2 a = lane < CL ? c.in2[lane] : Msg2{0.f, 0.f, 0.f, 0.f, 0ull, 0ull};
+            if (do_clip) {
+                g_clip_d = warp_sum(a.clip_d);
+                g_clip_q = warp_sum(a.clip_q);
+                g_n_clip = warp_sum(a.n_clip);
+            }
+            if (STOCH && do_sample) {
+                R = warp_sum_u64(a.mass);
+                before = warp_sum_u64(lane < static_cast<int>(rank) ? a.mass : 0ull) + wpre;
             }
         }
-        cluster_sync();  // #2
 
         // ------------------------------------------------ row results (every warp)
         float kc = 0.f, P = 0.f, Q = 0.f, Pc = 0.f, hardc = 0.f;
-        unsigned long long R = 0ull, before = 0ull;
-        {
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-            unsigned long long m = 0ull;
-            if (lane < CL) {
-                const uint32_t a = dsmem_map(&c.cta2, lane);
-                float v[4];
-                dsmem_ld4(a, v);
-                a0 = v[0]; a1 = v[1]; a2 = v[2];
-                m = dsmem_ld_u64(a + offsetof(Part2, mass));
-            }
-            R = warp_sum_u64(m);
-            before = warp_sum_u64(lane < static_cast<int>(rank) ? m : 0ull) + c.wpre[warp];
-            if (DISTILL && isRow) {
-                a0 = warp_sum(a0);
-                a1 = warp_sum(a1);
-                a2 = warp_sum(a2);
-                // S = sum over unclipped entries of q (s + 1) = (rkl - clip_d) + (1 - clip_q)
-                const float S = (rkl - a0) + (1.f - a1);
-                kc = isfinite(cc) ? (rkl - a0) + cc * a2 : rkl;
-                const float lam = p.lambda, pre = p.grad_scale * itau;
-                P = pre * (lam + (1.f - lam) * (1.f - S - dl));
-                Q = pre * (1.f - lam) * itau;
-                Pc = pre * (lam - (1.f - lam) * S);
-                hardc = pre * lam;
-            }
+        if (DISTILL && isRow) {
+            // S = sum over unclipped entries of q (s + 1) = (rkl - clip_d) + (1 - clip_q)
+            const float S = (rkl - g_clip_d) + (1.f - g_clip_q);
+            kc = isfinite(cc) ? (rkl - g_clip_d) + cc * g_n_clip : rkl;
+            const float lam = p.lambda, pre = p.grad_scale * itau;
+            P = pre * (lam + (1.f - lam) * (1.f - S - dl));
+            Q = pre * (1.f - lam) * itau;
+            Pc = pre * (lam - (1.f - lam) * S);
+            hardc = pre * lam;
         }
-        uint32_t y = kNone;
-        {
-            const uint32_t a = dsmem_map(dep0, 0);
-            uint32_t yv = 0, xv = 0;
-            if (lane == 0) {
-                yv = dsmem_ld_u32(a + offsetof(Deposit, argT));
-                if (rowVerify && p.draft == nullptr) xv = dsmem_ld_u32(a + offsetof(Deposit, argD));
-            }
-            y = __shfl_sync(0xffffffffu, yv, 0);
-            if (rowVerify && p.draft == nullptr) x = __shfl_sync(0xffffffffu, xv, 0);
-        }
-        if (rowVerify && !STOCH) acc = (x == y) ? 1 : 0;
 
-        // stochastic fallback: residual mass zero -> sample from p (rare; one more reduction)
+        // stochastic fallback: residual mass zero -> sample from p (rare; one more exchange)
         bool use_p = false;
         if (STOCH && do_sample && R == 0ull && isRow) {
             use_p = true;
+            if (t == 0) mbar_arrive_expect_tx(&c.x3, static_cast<uint32_t>(CL * sizeof(unsigned long long)));
             wmass = 0ull;
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
@@ -809,21 +906,22 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 wmass += ms;
             }
             wmass = warp_sum_u64(wmass);
-            if (lane == 0) c.p2[warp].mass = wmass;
+            __syncthreads();   // every warp is done with the exchange #2 partials
+            if (lane == 0) c.w2[warp].mass = wmass;
             __syncthreads();
+            const unsigned long long mw = lane < NW ? c.w2[lane].mass : 0ull;
+            const unsigned long long wpre = warp_prefix(mw);
             if (warp == 0) {
-                const unsigned long long m = lane < NW ? c.p2[lane].mass : 0ull;
-                unsigned long long incl = m;
-                warp_inclusive_scan_u64(incl);
-                if (lane < NW) c.wpre[lane] = incl - m;
-                const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
-                if (lane == 0) c.cta3.mass = tot;
+                const unsigned long long tot = warp_sum_u64(mw);
+                if (lane < CL)
+                    st_async_u64(dsmem_map(&c.in3[rank], static_cast<uint32_t>(lane)), tot,
+                                 dsmem_map(&c.x3, static_cast<uint32_t>(lane)));
             }
-            cluster_sync();
-            const unsigned long long m =
-                lane < CL ? dsmem_ld_u64(dsmem_map(&c.cta3, lane) + offsetof(Part2, mass)) : 0ull;
+            wait_x(&c.x3, n3 & 1u);
+            ++n3;
+            const unsigned long long m = lane < CL ? c.in3[lane] : 0ull;
             R = warp_sum_u64(m);
-            before = warp_sum_u64(lane < static_cast<int>(rank) ? m : 0ull) + c.wpre[warp];
+            before = warp_sum_u64(lane < static_cast<int>(rank) ? m : 0ull) + wpre;
         }
 
         // -------------------------------------------------------- sample search
@@ -860,67 +958,69 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                         }
                     }
                     if (pick < 0) pick = 7;
-                    dsmem_min_u32(dsmem_map(&dep0->tok, 0),
-                                  static_cast<uint32_t>(v0 + (wv0 + j * 32 + lane) * 8 + pick));
+                    atomicMin(&c.my_tok[par], static_cast<uint32_t>(v0 + (wv0 + j * 32 + lane) * 8 + pick));
                 }
             }
         }
 
         // -------------------------------------------------------- pass C: gradient row
         if (DISTILL && isRow) {
+            const float2 nL2D = make_float2(-L2D, -L2D), QQ = make_float2(Q, Q), PP = make_float2(P, P);
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
                 const int lv = j * 32 + lane;
-                float xd[8], xt[8], gv[8];
+                float2 xd[4], xt[4], g[4];
+                unpack8x2(myD[lv], xd);
+                unpack8x2(myT[lv], xt);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 a = fma2(xd[h], K2, nL2D);
+                    const float2 q = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+                    g[h] = mul2(q, fma2(QQ, sub2(xd[h], xt[h]), PP));
+                }
+                if (lv < wcnt) store_vec(drow, lv, g);
+            }
+            // vectors holding clipped entries are stored again with the clipped form
+            while (clipmask) {
+                const int j = __ffs(clipmask) - 1;
+                clipmask &= clipmask - 1u;
+                const int lv = j * 32 + lane;
+                float xd[8], xt[8];
                 unpack8(myD[lv], xd);
                 unpack8(myT[lv], xt);
+                float gl[8];
 #pragma unroll
                 for (int l = 0; l < 8; ++l) {
-                    const float q = fast_exp2(fmaf(xd[l], k2, -L2D));
-                    gv[l] = q * fmaf(Q, xd[l] - xt[l], P);
+                    const float q = elem_q(xd[l], k2, L2D);
+                    const float d = elem_d(q, elem_s(xd[l], xt[l], itau, dl));
+                    gl[l] = d > cc ? q * Pc : q * fmaf(Q, xd[l] - xt[l], P);
                 }
-                if (clipmask & (1u << j)) {
+                const float2 g[4] = {make_float2(gl[0], gl[1]), make_float2(gl[2], gl[3]),
+                                     make_float2(gl[4], gl[5]), make_float2(gl[6], gl[7])};
+                if (lv < wcnt) store_vec(drow, lv, g);
+            }
+            // the owner of y stores its entry again with the hard-label term and reports -log q_y
+            const int yl = static_cast<int>(y) - v0;
+            if (y != kNone && yl >= 0 && yl < len) {
+                const int vi = yl >> 3;
+                if (vi / vpw == warp) {
+                    const int lvy = vi - wv0;
+                    if ((lvy & 31) == lane) {
+                        float xd[8], xt[8];
+                        unpack8(myD[lvy], xd);
+                        unpack8(myT[lvy], xt);
+                        float dy = xd[0], ty = xt[0];
 #pragma unroll
-                    for (int l = 0; l < 8; ++l) {
-                        const float q = elem_q(xd[l], k2, L2D);
-                        const float d = elem_d(q, elem_s(xd[l], xt[l], itau, dl));
-                        if (d > cc) gv[l] = q * Pc;
-                    }
-                }
-                if (lv < wcnt) {
-                    const int base = v0 + (wv0 + lv) * 8;
-                    if (y >= static_cast<uint32_t>(base) && y < static_cast<uint32_t>(base + 8)) {
-                        const int ly = static_cast<int>(y) - base;
-                        float dy = xd[0];
-#pragma unroll
-                        for (int q = 1; q < 8; ++q) if (q == ly) dy = xd[q];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) if (q == ly) gv[q] -= hardc;
-                        // -log q_y = lseD - D_y / tau
-                        dsmem_st_f32(dsmem_map(&dep0->ce, 0), lseD - dy * itau);
-                    }
-                    if (ALIGNED) {
-                        if (p.dl_fp32) {
-                            float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.dlogits) + drow * V + base);
-                            __stcs(o, make_float4(gv[0], gv[1], gv[2], gv[3]));
-                            __stcs(o + 1, make_float4(gv[4], gv[5], gv[6], gv[7]));
-                        } else {
-                            uint4 pk;
-                            pk.x = pack_bf16x2(gv[0], gv[1]);
-                            pk.y = pack_bf16x2(gv[2], gv[3]);
-                            pk.z = pack_bf16x2(gv[4], gv[5]);
-                            pk.w = pack_bf16x2(gv[6], gv[7]);
-                            __stcs(reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dlogits) + drow * V + base), pk);
+                        for (int q = 1; q < 8; ++q)
+                            if (q == (yl & 7)) { dy = xd[q]; ty = xt[q]; }
+                        const float qa = fast_exp2(fmaf(dy, k2, -L2D));
+                        float gy = qa * fmaf(Q, dy - ty, P);
+                        if (do_clip) {
+                            const float q = elem_q(dy, k2, L2D);
+                            if (elem_d(q, elem_s(dy, ty, itau, dl)) > cc) gy = q * Pc;
                         }
-                    } else {
-#pragma unroll
-                        for (int l = 0; l < 8; ++l) {
-                            if (base + l < V && (wv0 + lv) * 8 + l < len) {
-                                if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + base + l] = gv[l];
-                                else static_cast<uint16_t*>(p.dlogits)[drow * V + base + l] =
-                                    static_cast<uint16_t>(pack_bf16x2(gv[l], 0.f) & 0xffffu);
-                            }
-                        }
+                        store_elem(drow, static_cast<int>(y), gy - hardc);
+                        c.my_ce[par] = lseD - dy * itau;   // -log q_y
                     }
                 }
             }
@@ -948,7 +1048,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         __syncwarp();
         if (ALIGNED && lane == 0 && nxt.kind != kItemNone) issue_loads(nxt);
 
-        // rank 0 keeps this row's values; the record is written after the next cluster barrier
+        // rank 0 keeps this row's values; the record is written after the next exchange #1
         if (rank == 0 && warp == NW - 1 && lane == 0) {
             Pending& pd = c.pend;
             pd.b = b; pd.i = i; pd.kind = cur.kind;
@@ -962,14 +1062,30 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             pd.kc = kc;
         }
         pending = true;
-        par ^= 1;
         cur = nxt;
         w = wn;
-        ++iter;
+        ++it;
     }
-    if (pending) {  // uniform: every rank walked the same items
-        cluster_sync();
-        if (rank == 0 && warp == NW - 1) write_record();
+    if (pending) {
+        // uniform: every rank walked the same items.  One more exchange #1 carries the last
+        // row's sampled token and -log q_y to rank 0.
+        const int par = it & 1;
+        if (t == 0) mbar_arrive_expect_tx(&c.x1[par], static_cast<uint32_t>(CL * sizeof(Msg1)));
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t ptok = c.my_tok[par ^ 1];
+            const float pce = c.my_ce[par ^ 1];
+            const uint32_t ninf = __float_as_uint(kNegInf);
+            send1(make_uint4(ninf, 0u, 0u, ninf), make_uint4(ninf, 0u, kNone, kNone),
+                  make_uint4(ptok, __float_as_uint(pce), 0u, 0u), par);
+        }
+        wait_x(&c.x1[par], static_cast<uint32_t>(it >> 1) & 1u);
+        if (rank == 0 && warp == NW - 1) {
+            const Msg1 a = lane < CL ? c.in1[par][lane] : empty_msg1();
+            const uint32_t ptok = redux_min_u32(a.prev_tok);
+            const float pce = warp_sum(a.prev_ce);
+            if (lane == 0) write_record(ptok, pce);
+        }
     }
 
     // ---------------------------------------------------------------- zero-only gradient rows
