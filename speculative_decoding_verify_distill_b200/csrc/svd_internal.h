@@ -124,7 +124,7 @@ int launch_wait_timeout_selftest(WsHeader* hdr, uint64_t limit_ns, void* stream)
 
 // Cluster geometry chosen for a vocabulary size.
 struct RowGeometry {
-    int variant;   // 0: 128 threads x 2 vectors; 1: 256 x 5; 2: 256 x 10
+    int variant;   // 0: 128 threads x 2 vectors per lane; 1: 256 x 10
     int threads;
     int cluster;   // CTAs per row
     int chunk;     // elements per CTA
