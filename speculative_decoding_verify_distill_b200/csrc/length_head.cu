@@ -65,8 +65,6 @@ __device__ __forceinline__ void stage_tile(uint16_t* dst, const uint16_t* src, i
 }  // namespace
 
 __global__ void __launch_bounds__(kWarps * 32) length_head_kernel(const HeadParams p) {
-    // let the dependent row pass start its prologue (it waits for this grid before reading b_k)
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ __align__(16) uint16_t hs[kHeadTileB * kLd];
     __shared__ __align__(16) uint16_t ws[kHeadTileM * kLd];
     __shared__ float pre[kHeadTileB][kHeadTileM + 1];

@@ -78,7 +78,7 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
                     uint64_t step, float lambda, float clip_c, float grad_scale, int dl_fp32,
                     void* dlogits, float* loss_rows, float* loss_total, int32_t* accept_len,
                     int32_t* emitted, int32_t* n_emitted, svd_row_info* row_info, const WsPtrs& w,
-                    void* stream, int pdl = 0) {
+                    void* stream) {
     RowParams p;
     std::memset(&p, 0, sizeof p);
     p.D = D; p.T = T; p.draft = draft; p.bk = bk;
@@ -97,7 +97,6 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
     p.row_info = row_info;
     p.hdr = w.hdr; p.rec = w.rec; p.seq_loss = w.seq_loss;
     p.wait_limit_ns = kWaitLimitNs;
-    p.pdl = pdl;
     return from_cuda(launch_row_pass(p, stream));
 }
 
@@ -215,7 +214,7 @@ svd_status svd_verify_distill(const svd_verify_distill_args* a, void* ws, size_t
     return run_rows(a->D, a->T, a->draft_tok, bk, a->B, a->k, a->kt, a->V, flags, a->temperature,
                     a->seed, a->step, a->lambda, a->clip_c, a->grad_scale, a->dlogits_fp32,
                     a->dlogits, a->loss_rows, a->loss_total, a->accept_len, a->emitted,
-                    a->n_emitted, a->row_info, w, stream, head ? 1 : 0);
+                    a->n_emitted, a->row_info, w, stream);
 }
 
 svd_status svd_get_device_error(void* ws, void* stream) {

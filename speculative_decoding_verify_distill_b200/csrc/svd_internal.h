@@ -114,7 +114,6 @@ struct RowParams {
     svd_row_info* rec;
     float* seq_loss;
     uint64_t wait_limit_ns;
-    int pdl;           // launched as a programmatic dependent of the length head
 };
 
 // Launchers (return cudaError_t as int; 0 = success).

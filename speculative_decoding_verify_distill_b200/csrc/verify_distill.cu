@@ -11,8 +11,8 @@
 // zero gradient row.
 //
 // Design (B200, sm_100a):
-//   * A persistent grid of thread-block clusters (8 CTAs of 256 threads for a 151936-id
-//     vocabulary, two CTAs per SM).  A cluster owns one logit row at a time; each CTA a
+//   * A persistent grid of thread-block clusters (10 CTAs of 256 threads for a 151936-id
+//     vocabulary, three CTAs per SM).  A cluster owns one logit row at a time; each CTA a
 //     contiguous slice of the vocabulary; each warp a contiguous run of 16-byte vectors of the
 //     slice.  Loaded work items (verified rows and bonus rows) form a compact list (prefix sums
 //     of loaded rows per sequence) handed out one row at a time from a workspace ticket, so a
@@ -325,9 +325,6 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         }
     }
     __syncthreads();
-    // behind the length head (programmatic dependent launch) the prologue above overlapped its
-    // tail; b_k is read only after the head's writes are visible
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     const bool compact = p.B <= kCompactMaxB;
     if (compact) {
         // b_k and the exclusive prefixes of loaded rows and zero-gradient rows per sequence
@@ -1273,12 +1270,14 @@ KernelFn pick_kernel(int flags, bool aligned) {
 }
 
 // Variants: (threads, vectors per lane, min CTAs per SM) -> ids per CTA = 8 * NT * NV.
-// Large vocabularies take few, long slices per row (8 CTAs at V = 151936, two CTAs per SM):
-// the per-row exchange is shared by more elements per thread.  Measured at B = 128, k = 16,
-// V = 151936 on B200: 0.404 ms per row pass, against 0.438 ms for 16 CTAs of 256 x 5 (four
-// per SM) and 0.450 ms for 4 CTAs of 512 x 10 (one per SM).
+// Large vocabularies: clusters of ceil(V / 16384) CTAs of 256 threads x 8 vectors, three CTAs
+// per SM (10 CTAs per row at V = 151936).  Measured at B = 128, k = 16, V = 151936 on B200, row
+// pass alone: 0.365 ms, against 0.405 ms for 8 CTAs of 256 x 10 (two per SM), 0.438 ms for 16
+// of 256 x 5 (four per SM), 0.431 ms for 11 of 256 x 7 and 0.450 ms for 4 of 512 x 10.
+// Vocabularies whose slices would need more than 16 CTAs take 256 x 10.
 constexpr int kSNT = 128, kSNV = 2, kSMB = 8;     //  2048 ids per CTA
-constexpr int kLNT = 256, kLNV = 10, kLMB = 2;    // 20480 ids per CTA
+constexpr int kLNT = 256, kLNV = 8, kLMB = 3;     // 16384 ids per CTA
+constexpr int kXNT = 256, kXNV = 10, kXMB = 2;    // 20480 ids per CTA
 
 int next_pow2(int x) {
     int r = 1;
@@ -1290,15 +1289,19 @@ int next_pow2(int x) {
 
 bool row_geometry(int V, RowGeometry* g) {
     if (V < 1) return false;
-    const int capS = kSNT * kSNV * 8, capL = kLNT * kLNV * 8;
+    const int capS = kSNT * kSNV * 8, capL = kLNT * kLNV * 8, capX = kXNT * kXNV * 8;
     if (V <= 8 * capS) {
         g->variant = 0; g->threads = kSNT;
         g->cluster = next_pow2((V + capS - 1) / capS);
         g->smem = smem_fixed<kSNT, kSNV>();
-    } else {
+    } else if (V <= 16 * capL) {
         g->variant = 1; g->threads = kLNT;
-        g->cluster = next_pow2((V + capL - 1) / capL);
+        g->cluster = (V + capL - 1) / capL;
         g->smem = smem_fixed<kLNT, kLNV>();
+    } else {
+        g->variant = 2; g->threads = kXNT;
+        g->cluster = (V + capX - 1) / capX;
+        g->smem = smem_fixed<kXNT, kXNV>();
     }
     if (g->cluster > 16) return false;
     const int per = (V + g->cluster - 1) / g->cluster;
@@ -1317,7 +1320,8 @@ int launch_row_pass(const RowParams& p, void* stream) {
     if (!row_geometry(p.V, &geo)) return static_cast<int>(cudaErrorInvalidValue);
     const bool aligned = p.aligned != 0;
     KernelFn fn = geo.variant == 0 ? pick_kernel<kSNT, kSNV, kSMB>(p.flags, aligned)
-                                   : pick_kernel<kLNT, kLNV, kLMB>(p.flags, aligned);
+                : geo.variant == 1 ? pick_kernel<kLNT, kLNV, kLMB>(p.flags, aligned)
+                                   : pick_kernel<kXNT, kXNV, kXMB>(p.flags, aligned);
     const size_t smem = row_smem_bytes(geo, p.B);
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
@@ -1327,24 +1331,19 @@ int launch_row_pass(const RowParams& p, void* stream) {
         if (err != cudaSuccess) return static_cast<int>(err);
     }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = geo.cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (p.pdl) {
-        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[1].val.programmaticStreamSerializationAllowed = 1;
-        cfg.numAttrs = 2;
-    }
     cfg.blockDim = dim3(geo.threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
     // persistent grid: as many clusters as can be resident at once (cached per configuration)
-    static int cached_clusters[2][17][8][2] = {};
-    static size_t cached_smem[2][17][8][2] = {};
+    static int cached_clusters[3][17][8][2] = {};
+    static size_t cached_smem[3][17][8][2] = {};
     int& cache = cached_clusters[geo.variant][geo.cluster][p.flags & 7][aligned ? 1 : 0];
     size_t& csm = cached_smem[geo.variant][geo.cluster][p.flags & 7][aligned ? 1 : 0];
     if (cache == 0 || csm != smem) {

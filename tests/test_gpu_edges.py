@@ -54,7 +54,8 @@ def full_compare(vd, D, T, bk, *, draft=None, mode=0, tau=1.0, lam=0.5, clip_c=1
     return st
 
 
-@pytest.mark.parametrize("V", [1, 7, 8, 9, 1000, 1024, 1031, 4104, 16384, 16392, 40960])
+@pytest.mark.parametrize("V", [1, 7, 8, 9, 1000, 1024, 1031, 4104, 16384, 16392, 40960, 100000,
+                               200003, 262144, 262152, 327680])
 def test_vocab_sizes_greedy(V):
     B, k = 3, 4
     D, T = make_case(B, k, k, V, seed=V)
