@@ -17,8 +17,8 @@
 //     slice.  Loaded work items (verified rows and bonus rows) form a compact list (prefix sums
 //     of loaded rows per sequence) handed out one row at a time from a workspace ticket, so a
 //     cluster that starts late (behind the length head, or beside other work) simply takes fewer
-//     rows.  Zero-only gradient rows follow, in quarter-row units handed out to single CTAs,
-//     without cluster barriers.
+//     rows.  Zero-only gradient rows are handed to single CTAs in sixteenth-row units: one per
+//     CTA while each row's exchange is in flight, the rest after the loaded rows.
 //   * Each warp stages its run of D and T in shared memory with its own 1-D bulk copies
 //     (cp.async.bulk, no multicast) on its own mbarrier.  The staged bf16 slice is the only copy:
 //     every pass re-reads it, so a CTA holds no per-element state in registers and several CTAs
@@ -93,14 +93,16 @@ struct Ctl {
     int wscanz[NW];                 // ... and of the zero-gradient row counts
     uint32_t first_item;            // rank 0: the cluster's first loaded item (packed)
     int zs;                         // zero phase: the CTA's next unit
+    int zu[2];                      // zero unit written while exchange #1 of a row is in flight
 };
 
 // Batches up to this size keep b_k and the prefixes of loaded and zero-gradient rows per sequence
 // in shared memory (compact lists, handed out dynamically); larger batches walk the uncompacted
 // (sequence, row) slots in a fixed order.
 constexpr int kCompactMaxB = 4096;
-// Zero-gradient rows are handed out in quarters (about 75 KB of stores each at V = 151936).
-constexpr int kZeroSplit = 4;
+// Zero-gradient rows are handed out in sixteenths (about 19 KB of bf16 stores at V = 151936):
+// one unit per CTA fills the wait for each row's exchange, the rest follow the loaded rows.
+constexpr int kZeroSplit = 16;
 
 struct Item {
     int kind, b, i;
@@ -435,6 +437,36 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         else static_cast<uint16_t*>(p.dlogits)[drow * V + id] = static_cast<uint16_t>(pack_bf16x2(g, 0.f) & 0xffffu);
     };
 
+    // unit u of the compact zero-row list: a sixteenth of gradient row (b, i), i past b_k
+    const int zunits = (DISTILL && compact) ? zpre[p.B] * kZeroSplit : 0;
+    auto write_zero_unit = [&](int u) {
+        const int j = u / kZeroSplit, qq = u % kZeroSplit;
+        int lo = 0, hi = p.B;  // largest b with zpre[b] <= j
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (zpre[mid] <= j) lo = mid; else hi = mid;
+        }
+        const int i = first_zero_row(sbk[lo], verify) + (j - zpre[lo]);
+        const size_t drow = static_cast<size_t>(lo) * k + i;
+        if (ALIGNED) {
+            const uint4 zz = make_uint4(0, 0, 0, 0);
+            const int per_elem = p.dl_fp32 ? 2 : 1;       // 16-byte stores per 8 ids
+            const int nv = (V / 8) * per_elem;
+            const int a0 = static_cast<int>(static_cast<long long>(nv) * qq / kZeroSplit);
+            const int a1 = static_cast<int>(static_cast<long long>(nv) * (qq + 1) / kZeroSplit);
+            uint4* g = p.dl_fp32 ? reinterpret_cast<uint4*>(static_cast<float*>(p.dlogits) + drow * V)
+                                 : reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dlogits) + drow * V);
+            for (int e = a0 + t; e < a1; e += NT) __stcs(g + e, zz);
+        } else {
+            const int a0 = static_cast<int>(static_cast<long long>(V) * qq / kZeroSplit);
+            const int a1 = static_cast<int>(static_cast<long long>(V) * (qq + 1) / kZeroSplit);
+            for (int e = a0 + t; e < a1; e += NT) {
+                if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + e] = 0.f;
+                else static_cast<uint16_t*>(p.dlogits)[drow * V + e] = 0;
+            }
+        }
+    };
+
     Item cur{kItemNone, -1, -1};
     int w = cid;
     if (compact) {
@@ -500,6 +532,9 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         // rank 0 asks for the next item now; it travels in this row's message #1
         uint32_t fetched = 0;
         if (compact && rank == 0 && t == 0) fetched = atomicAdd(&p.hdr->item_ticket, 1u);
+        // and every CTA asks for one zero-row unit to write while this row's exchange is in flight
+        int zfetch = 0;
+        if (zunits > 0 && t == 0) zfetch = static_cast<int>(atomicAdd(&p.hdr->zero_ticket, 1u));
         if (t == 0) mbar_arrive_expect_tx(&c.x1[par], static_cast<uint32_t>(CL * sizeof(Msg1)));
         const int b = cur.b, i = cur.i;
         const size_t drow = static_cast<size_t>(b) * k + i;      // draft / gradient row
@@ -660,6 +695,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             m.pad = 0u;
             if (lane == 0) c.w1[warp] = m;
         }
+        if (zunits > 0 && t == 0) c.zu[par] = zfetch;
         __syncthreads();
         if (warp == 0) {
             const Msg1 a = lane < NW ? c.w1[lane] : empty_msg1();
@@ -693,6 +729,10 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 c.my_tok[par ^ 1] = kNone;
                 c.my_ce[par ^ 1] = 0.f;
             }
+        }
+        if (zunits > 0) {
+            const int zu = c.zu[par];
+            if (zu < zunits) write_zero_unit(zu);
         }
         wait_x(&c.x1[par], static_cast<uint32_t>(it >> 1) & 1u);
 
@@ -1087,9 +1127,9 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
 
     // ---------------------------------------------------------------- zero-only gradient rows
     if (DISTILL && compact) {
-        // quarters of the zero rows in the compact list, handed to CTAs one at a time (the next
-        // unit is requested while the current one is written)
-        const int units = zpre[p.B] * kZeroSplit;
+        // the zero-row units not yet taken, handed to CTAs one at a time (the next unit is
+        // requested while the current one is written)
+        const int units = zunits;
         if (t == 0) c.zs = static_cast<int>(atomicAdd(&p.hdr->zero_ticket, 1u));
         __syncthreads();
         int u = c.zs;
@@ -1097,31 +1137,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         while (u < units) {
             int nextu = 0;
             if (t == 0) nextu = static_cast<int>(atomicAdd(&p.hdr->zero_ticket, 1u));
-            const int j = u / kZeroSplit, qq = u % kZeroSplit;
-            int lo = 0, hi = p.B;  // largest b with zpre[b] <= j
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (zpre[mid] <= j) lo = mid; else hi = mid;
-            }
-            const int i = first_zero_row(sbk[lo], verify) + (j - zpre[lo]);
-            const size_t drow = static_cast<size_t>(lo) * k + i;
-            if (ALIGNED) {
-                const uint4 zz = make_uint4(0, 0, 0, 0);
-                const int per_elem = p.dl_fp32 ? 2 : 1;       // 16-byte stores per 8 ids
-                const int nv = (V / 8) * per_elem;
-                const int a0 = static_cast<int>(static_cast<long long>(nv) * qq / kZeroSplit);
-                const int a1 = static_cast<int>(static_cast<long long>(nv) * (qq + 1) / kZeroSplit);
-                uint4* g = p.dl_fp32 ? reinterpret_cast<uint4*>(static_cast<float*>(p.dlogits) + drow * V)
-                                     : reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dlogits) + drow * V);
-                for (int e = a0 + t; e < a1; e += NT) __stcs(g + e, zz);
-            } else {
-                const int a0 = static_cast<int>(static_cast<long long>(V) * qq / kZeroSplit);
-                const int a1 = static_cast<int>(static_cast<long long>(V) * (qq + 1) / kZeroSplit);
-                for (int e = a0 + t; e < a1; e += NT) {
-                    if (p.dl_fp32) static_cast<float*>(p.dlogits)[drow * V + e] = 0.f;
-                    else static_cast<uint16_t*>(p.dlogits)[drow * V + e] = 0;
-                }
-            }
+            write_zero_unit(u);
             if (t == 0) c.zs = nextu;
             __syncthreads();
             u = c.zs;
