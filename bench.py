@@ -292,6 +292,8 @@ def main():
     bk_host = bk.cpu().numpy()
     acc_host = fused.accept_len.cpu().numpy()
     ne_host = fused.n_emitted.cpu().numpy()
+    # the step's speedup report (rho = 0: verification-count view of the pages' eta)
+    report = api.report_dict(api.svd_speedup_report(fused.accept_len, bk, fused.n_emitted, w.k, 0.0))
 
     # ---------------------------------------------------------------- timed region (device)
     K = args.steps
@@ -410,6 +412,8 @@ def main():
             "step_hbm_gbs": (alg + head_bytes(w.B, w.H, w.M)) * info.world / (red["ms"] / 1000.0) / 1e9,
             "length_head_avg_ms": statistics.mean(head_ms),
             "bk_hist": bk_hist,
+            "speedup_report": {k_: (None if v_ != v_ else round(v_, 6)) for k_, v_ in report.items()
+                               if k_ != "alpha"},
         }
         print(json.dumps(line), flush=True)
     if info.world > 1:

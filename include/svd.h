@@ -164,6 +164,18 @@ typedef struct svd_verify_distill_args {
     float* loss_total;       /* [1]                                     */
     void* dlogits;           /* [B,k,V] bf16 / fp32                     */
     svd_row_info* row_info;  /* [B,kt] or NULL                          */
+    /* Length-head labels.  The head's online update fits bhat to an acceptance label a*; under
+     * truncated verification only a/b_k is observable (Pith verdict record, load_bearing_attack),
+     * and its proposed test (concrete_test; the review page's falsifier) verifies all k drafts to
+     * obtain the full-block label a/k.  full_k = 1 runs that variant: b_k (the head's choice, or
+     * bk_in) is still computed and written to `bk`, but every sequence verifies and distills all
+     * k rows; accept_len, emitted, n_emitted, the losses and the gradient are those of the
+     * full-k pass.  Acceptance is a prefix scan and each decision depends only on its own row,
+     * so min(a, b_k) is exactly the acceptance truncated verification would have seen. */
+    int full_k;              /* 0 or 1                                                        */
+    float* label_proxy;      /* [B] or NULL: a / b_k as truncated verification observes it;
+                              * with full_k = 1, min(a, b_k) / b_k                            */
+    float* label_full;       /* [B] or NULL: a / k with full_k = 1; NaN with full_k = 0         */
 } svd_verify_distill_args;
 
 /* a1 .. a5 in one call: the length head (unless h == NULL), then one persistent pass over the
@@ -202,6 +214,22 @@ svd_status svd_verify_distill(const svd_verify_distill_args* args, void* ws, siz
  * of 64 or more. */
 svd_status svd_verify_distill_noalloc(const svd_verify_distill_args* args, uint32_t* status_out,
                                       void* stream);
+
+/* Speedup reporter for one verification step (Pith review page, Referee Report minor comment 1,
+ * their Eq. 1: E[tau] = (1 - Acc^(k+1)) / (1 - Acc), eta = E[tau] / (rho*k + 1), which assumes
+ * i.i.d. acceptance; the measured values are reported beside the model).  Inputs are the
+ * step's outputs per sequence: accept_len a_b, bk n_b (rows verified) and n_emitted e_b, with
+ * 0 <= a_b <= n_b <= k.  `rho` is the drafter-to-target cost ratio of the speedup formula.
+ * Writes out [8 + k] fp64 (device):
+ *   out[0] measured E[tau] = mean e_b (tokens per target verification)
+ *   out[1] Acc = sum a_b / sum min(a_b + 1, n_b) (accepted / decisions taken)
+ *   out[2] model E[tau] from Acc; out[3] eta = out[2] / (rho*k + 1); out[4] = out[0] / (rho*k + 1)
+ *   out[5] mean n_b, out[6] mean a_b, out[7] B
+ *   out[8 + i] acceptance at position i given an accepted prefix and a verified row:
+ *              #{a_b > i} / #{a_b >= i and n_b > i} (NaN if no sequence reached row i). */
+svd_status svd_speedup_report(const int32_t* accept_len, const int32_t* bk,
+                              const int32_t* n_emitted, int B, int k, double rho, double* out,
+                              void* stream);
 
 /* Reads and clears the device status word of `ws` (synchronizes `stream`).  Returns SVD_OK,
  * SVD_ERR_TOKEN_RANGE or SVD_ERR_TIMEOUT as recorded by kernels that used this workspace, or

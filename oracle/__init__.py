@@ -14,6 +14,8 @@ Which pins hold each function (see ``tests/test_oracle_*.py``):
   * ``distill``      -- KL = 0 when draft == target; RKL >= 0; K_c <= RKL; c = inf equals torch
                         kl_div; lambda = 1 equals torch cross_entropy; a hand-derived V = 2
                         golden case; finite differences; torch autograd; sum of gradient = 0.
+  * ``speedup_report`` -- hand-counted small cases; all-accepted and all-rejected limits; the
+                        closed form recovered from geometric accept lengths (i.i.d. rate A).
   * ``philox``       -- parity unpinned against published known-answer vectors (none are
                         available offline); held by uniformity / independence chi-square tests
                         and by bit-exact agreement with the independent CUDA implementation.
@@ -58,6 +60,8 @@ def _load():
     lib.orc_length_head.argtypes = [P, P, P, P, f64, i32, i32, i32, i32, f64, i32, P, P, P]
     lib.orc_length_head.restype = i32
     lib.orc_row_stats.argtypes = [P, i32, f64, P, P, P]
+    lib.orc_speedup_report.argtypes = [P, P, P, i32, i32, f64, P]
+    lib.orc_speedup_report.restype = i32
     lib.orc_verify.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, f64, u64, u64,
                                P, P, P, P, P, P, P, P, P]
     lib.orc_verify.restype = i32
@@ -217,3 +221,18 @@ def distill(D, T, bk, lam: float, clip_c: float, tau: float = 1.0, grad_scale: f
 
 def expected_tokens(A: float, k: int) -> float:
     return float(_load().orc_expected_tokens(float(A), int(k)))
+
+
+def speedup_report(accept_len, bk, n_emitted, k: int, rho: float) -> np.ndarray:
+    """fp64 [8 + k]: measured E[tau], Acc, model E[tau], eta (model), eta (measured), mean b_k,
+    mean accepted length, B, then the per-position acceptance rates (see svd_oracle.c)."""
+    lib = _load()
+    a = np.ascontiguousarray(accept_len, np.int32)
+    n = np.ascontiguousarray(bk, np.int32)
+    e = np.ascontiguousarray(n_emitted, np.int32)
+    out = np.zeros(8 + int(k), np.float64)
+    rc = lib.orc_speedup_report(a.ctypes.data, n.ctypes.data, e.ctypes.data, len(a), int(k),
+                                float(rho), out.ctypes.data)
+    if rc != 0:
+        raise ValueError("orc_speedup_report: bad arguments")
+    return out

@@ -498,3 +498,48 @@ double orc_expected_tokens(double A, int k) {
     if (A == 1.0) return (double)(k + 1);
     return (1.0 - pow(A, (double)(k + 1))) / (1.0 - A);
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Speedup reporter for one verification step of B sequences ([PR] Referee minor comment 1,   */
+/* their Eq. 1, and the Axiom ledger's standard acceptance formula).  Inputs per sequence:     */
+/* accepted length a_b, verified rows n_b (= b_k) and emitted tokens e_b.                     */
+/*   out[0] measured E[tau] = mean_b e_b          (tokens per target verification)             */
+/*   out[1] Acc = sum_b a_b / sum_b t_b, where t_b = min(a_b + 1, n_b) is the number of rows    */
+/*          whose decision was taken (the accepted prefix and, if a_b < n_b, the rejected row) */
+/*   out[2] model E[tau] = (1 - Acc^(k+1)) / (1 - Acc) (i.i.d. acceptance; k + 1 at Acc = 1)    */
+/*   out[3] eta from the model = out[2] / (rho*k + 1)                                           */
+/*   out[4] eta from the measurement = out[0] / (rho*k + 1)                                     */
+/*   out[5] mean n_b, out[6] mean a_b, out[7] B                                                 */
+/*   out[8+i], i < k: alpha_i = #{b: a_b > i} / #{b: a_b >= i and n_b > i}, the acceptance at    */
+/*          position i given an accepted prefix and a verified row (NaN if no sequence got there)*/
+/* ------------------------------------------------------------------------------------------ */
+int orc_speedup_report(const int32_t* accept_len, const int32_t* bk, const int32_t* n_emitted,
+                       int B, int k, double rho, double* out) {
+    if (B < 1 || k < 1) return 1;
+    double sum_e = 0.0, sum_a = 0.0, sum_t = 0.0, sum_n = 0.0;
+    for (int b = 0; b < B; ++b) {
+        const int a = accept_len[b], n = bk[b];
+        sum_e += (double)n_emitted[b];
+        sum_a += (double)a;
+        sum_n += (double)n;
+        sum_t += (double)(a + 1 < n ? a + 1 : n);
+    }
+    const double acc = sum_t > 0.0 ? sum_a / sum_t : NAN;
+    out[0] = sum_e / (double)B;
+    out[1] = acc;
+    out[2] = orc_expected_tokens(acc, k);
+    out[3] = out[2] / (rho * (double)k + 1.0);
+    out[4] = out[0] / (rho * (double)k + 1.0);
+    out[5] = sum_n / (double)B;
+    out[6] = sum_a / (double)B;
+    out[7] = (double)B;
+    for (int i = 0; i < k; ++i) {
+        long accepted = 0, tested = 0;
+        for (int b = 0; b < B; ++b) {
+            if (accept_len[b] > i) ++accepted;
+            if (accept_len[b] >= i && bk[b] > i) ++tested;
+        }
+        out[8 + i] = tested > 0 ? (double)accepted / (double)tested : NAN;
+    }
+    return 0;
+}

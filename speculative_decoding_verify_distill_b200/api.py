@@ -51,6 +51,7 @@ class VerifyDistillArgs(ctypes.Structure):
         ("lambda_", _F), ("clip_c", _F), ("grad_scale", _F), ("dlogits_fp32", _I),
         ("bhat", _P), ("bk", _P), ("accept_len", _P), ("emitted", _P), ("n_emitted", _P),
         ("loss_rows", _P), ("loss_total", _P), ("dlogits", _P), ("row_info", _P),
+        ("full_k", _I), ("label_proxy", _P), ("label_full", _P),
     ]
 
 
@@ -80,9 +81,10 @@ def lib():
     L.svd_status_string.restype = ctypes.c_char_p
     L.svd_selftest_wait_timeout.argtypes = [_P, _SZ, _U64, _P]
     L.svd_verify_distill_noalloc.argtypes = [ctypes.POINTER(VerifyDistillArgs), _P, _P]
+    L.svd_speedup_report.argtypes = [_P, _P, _P, _I, _I, ctypes.c_double, _P, _P]
     for fn in ("svd_workspace_reset", "svd_length_head", "svd_verify", "svd_distill_loss_grad",
                "svd_verify_distill", "svd_get_device_error", "svd_selftest_wait_timeout",
-               "svd_verify_distill_noalloc"):
+               "svd_verify_distill_noalloc", "svd_speedup_report"):
         getattr(L, fn).restype = _I
     _lib = L
     return L
@@ -227,7 +229,8 @@ class VerifyDistill:
 
     def __init__(self, D, T, *, head=None, bk_in=None, draft_tok=None, mode=GREEDY,
                  temperature=1.0, seed=0, step=0, lam=0.5, clip_c=1.0, grad_scale=1.0,
-                 gamma=1.0, rnd=BK_CEIL, dlogits_fp32=False, row_info=False, ws=None):
+                 gamma=1.0, rnd=BK_CEIL, dlogits_fp32=False, row_info=False, ws=None,
+                 full_k=False, labels=False):
         B, k, V = D.shape
         kt = T.shape[1]
         dev = D.device
@@ -244,6 +247,9 @@ class VerifyDistill:
         self.dlogits = torch.empty((B, k, V), dtype=torch.float32 if dlogits_fp32 else torch.bfloat16,
                                    device=dev)
         self.row_info = _row_info_tensor(B, kt, dev) if row_info else None
+        # length-head labels: a / b_k as truncated verification sees it, and a / k (full-k mode)
+        self.label_proxy = torch.empty(B, dtype=torch.float32, device=dev) if labels else None
+        self.label_full = torch.empty(B, dtype=torch.float32, device=dev) if labels else None
         a = VerifyDistillArgs()
         if head is not None:
             h, W1, b1, w2, b2 = head
@@ -263,6 +269,8 @@ class VerifyDistill:
         a.accept_len, a.emitted, a.n_emitted = _ptr(self.accept_len), _ptr(self.emitted), _ptr(self.n_emitted)
         a.loss_rows, a.loss_total, a.dlogits = _ptr(self.loss_rows), _ptr(self.loss_total), _ptr(self.dlogits)
         a.row_info = _ptr(self.row_info)
+        a.full_k = int(bool(full_k))
+        a.label_proxy, a.label_full = _ptr(self.label_proxy), _ptr(self.label_full)
         self.args = a
 
     def set_step(self, step: int):
@@ -279,12 +287,36 @@ class VerifyDistill:
                    dlogits=self.dlogits)
         if self.row_info is not None:
             out["row_info"] = self.row_info
+        if self.label_proxy is not None:
+            out["label_proxy"] = self.label_proxy
+            out["label_full"] = self.label_full
         return out
 
 
 def svd_verify_distill(D, T, **kw) -> dict:
     """a1-a5 in one call; keyword arguments as in :class:`VerifyDistill`."""
     return VerifyDistill(D, T, **kw)().outputs()
+
+
+REPORT_FIELDS = ("tau_measured", "acc", "tau_model", "eta_model", "eta_measured", "mean_bk",
+                 "mean_accept", "B")
+
+
+def svd_speedup_report(accept_len, bk, n_emitted, k: int, rho: float = 0.0, stream=None):
+    """E[tau] (measured and modelled), Acc, eta and per-position acceptance as a fp64 CUDA
+    tensor [8 + k]; see :func:`report_dict` for the field names."""
+    out = torch.empty(8 + int(k), dtype=torch.float64, device=accept_len.device)
+    _check(lib().svd_speedup_report(_ptr(accept_len), _ptr(bk), _ptr(n_emitted),
+                                    int(accept_len.numel()), int(k), float(rho), _ptr(out),
+                                    _stream(stream)), "svd_speedup_report")
+    return out
+
+
+def report_dict(out) -> dict:
+    v = out.double().cpu().tolist()
+    d = dict(zip(REPORT_FIELDS, v[:8]))
+    d["alpha"] = v[8:]
+    return d
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20

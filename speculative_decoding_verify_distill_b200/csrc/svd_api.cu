@@ -78,7 +78,8 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
                     uint64_t step, float lambda, float clip_c, float grad_scale, int dl_fp32,
                     void* dlogits, float* loss_rows, float* loss_total, int32_t* accept_len,
                     int32_t* emitted, int32_t* n_emitted, svd_row_info* row_info, const WsPtrs& w,
-                    void* stream) {
+                    void* stream, int bk_const = 0, float* label_proxy = nullptr,
+                    float* label_full = nullptr) {
     RowParams p;
     std::memset(&p, 0, sizeof p);
     p.D = D; p.T = T; p.draft = draft; p.bk = bk;
@@ -97,6 +98,10 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
     p.row_info = row_info;
     p.hdr = w.hdr; p.rec = w.rec; p.seq_loss = w.seq_loss;
     p.wait_limit_ns = kWaitLimitNs;
+    p.bk_const = bk_const;
+    p.bk_trunc = bk;
+    p.label_proxy = label_proxy;
+    p.label_full = label_full;
     return from_cuda(launch_row_pass(p, stream));
 }
 
@@ -183,6 +188,7 @@ svd_status svd_verify_distill(const svd_verify_distill_args* a, void* ws, size_t
     if (bad_float(a->lambda) || a->lambda < 0.f || a->lambda > 1.f) return SVD_ERR_INVALID_ARG;
     if (std::isnan(a->clip_c) || a->clip_c < 0.f || bad_float(a->grad_scale)) return SVD_ERR_INVALID_ARG;
     if (a->dlogits_fp32 != 0 && a->dlogits_fp32 != 1) return SVD_ERR_INVALID_ARG;
+    if (a->full_k != 0 && a->full_k != 1) return SVD_ERR_INVALID_ARG;
     const bool head = a->h != nullptr;
     if (head) {
         if (a->H < 1 || a->M < 1 || !a->W1 || !a->w2) return SVD_ERR_INVALID_ARG;
@@ -214,7 +220,16 @@ svd_status svd_verify_distill(const svd_verify_distill_args* a, void* ws, size_t
     return run_rows(a->D, a->T, a->draft_tok, bk, a->B, a->k, a->kt, a->V, flags, a->temperature,
                     a->seed, a->step, a->lambda, a->clip_c, a->grad_scale, a->dlogits_fp32,
                     a->dlogits, a->loss_rows, a->loss_total, a->accept_len, a->emitted,
-                    a->n_emitted, a->row_info, w, stream);
+                    a->n_emitted, a->row_info, w, stream, a->full_k ? a->k : 0, a->label_proxy,
+                    a->label_full);
+}
+
+svd_status svd_speedup_report(const int32_t* accept_len, const int32_t* bk,
+                              const int32_t* n_emitted, int B, int k, double rho, double* out,
+                              void* stream) {
+    if (B < 1 || k < 1 || k > kMaxK || !std::isfinite(rho) || rho < 0.0) return SVD_ERR_INVALID_ARG;
+    if (!accept_len || !bk || !n_emitted || !out) return SVD_ERR_INVALID_ARG;
+    return from_cuda(launch_speedup_report(accept_len, bk, n_emitted, B, k, rho, out, stream));
 }
 
 svd_status svd_get_device_error(void* ws, void* stream) {

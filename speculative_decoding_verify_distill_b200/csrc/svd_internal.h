@@ -114,12 +114,18 @@ struct RowParams {
     svd_row_info* rec;
     float* seq_loss;
     uint64_t wait_limit_ns;
+    int bk_const;                // > 0: every sequence verifies this many rows (full-k mode)
+    const int32_t* bk_trunc;     // the truncated choice of b_k, for the labels
+    float* label_proxy;          // [B] or null
+    float* label_full;           // [B] or null
 };
 
 // Launchers (return cudaError_t as int; 0 = success).
 int launch_length_head(const HeadParams& p, void* stream);
 int launch_row_pass(const RowParams& p, void* stream);
 int launch_wait_timeout_selftest(WsHeader* hdr, uint64_t limit_ns, void* stream);
+int launch_speedup_report(const int32_t* accept_len, const int32_t* bk, const int32_t* n_emitted,
+                          int B, int k, double rho, double* out, void* stream);
 
 // Cluster geometry chosen for a vocabulary size.
 struct RowGeometry {

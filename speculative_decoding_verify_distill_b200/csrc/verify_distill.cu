@@ -168,12 +168,15 @@ __device__ __forceinline__ int zero_rows(int k, int n, bool verify) {
 }
 __device__ __forceinline__ int first_zero_row(int n, bool verify) { return verify ? n + 1 : n; }
 
-// b_k of sequence b: from shared memory (compact mode) or global memory (clamped).
+// Rows sequence b verifies: all k in full-k mode, else its b_k (clamped).
+__device__ __forceinline__ int load_bk(const RowParams& p, int b) {
+    return p.bk_const > 0 ? p.bk_const : clamp_bk(p, __ldg(p.bk + b));
+}
+// b_k of sequence b: from shared memory (compact mode) or global memory.
 struct BkView {
     const int* s;       // shared copy, or nullptr
-    const int32_t* g;   // global
     __device__ __forceinline__ int operator()(const RowParams& p, int b) const {
-        return s ? s[b] : clamp_bk(p, __ldg(g + b));
+        return s ? s[b] : load_bk(p, b);
     }
 };
 
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             const int b = c0 + t;
             int n = 0, L = 0, Z = 0;
             if (b < p.B) {
-                n = clamp_bk(p, __ldg(p.bk + b));
+                n = load_bk(p, b);
                 L = loaded_rows(n, kt, verify);
                 Z = DISTILL ? zero_rows(k, n, verify) : 0;
                 sbk[b] = n;
@@ -370,14 +373,14 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             // rank 0 takes the cluster's first loaded item from the workspace ticket
             if (rank == 0) {
                 const int w0 = static_cast<int>(atomicAdd(&p.hdr->item_ticket, 1u));
-                c.first_item = pack_item(decode_loaded(p, spre, BkView{sbk, p.bk}, w0, verify));
+                c.first_item = pack_item(decode_loaded(p, spre, BkView{sbk}, w0, verify));
             }
         }
     }
     __syncthreads();
     cluster_sync();  // barriers, lists and the first item ready everywhere
 
-    const BkView bkv{compact ? sbk : nullptr, p.bk};
+    const BkView bkv{compact ? sbk : nullptr};
     const int* list = compact ? spre : nullptr;
     const int nslots = loaded_slots(p, list);
     // Compact mode: rank 0 takes loaded items one at a time from the workspace ticket, one row
@@ -1189,7 +1192,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(const RowParams p) {
     const int k = p.k, kt = p.kt;
     const int b = blockIdx.x * 8 + warp;
     if (b < p.B) {
-        int n = __ldg(p.bk + b);
+        int n = p.bk_const > 0 ? p.bk_const : __ldg(p.bk + b);
         n = n < 1 ? 1 : (n > k ? k : n);   // the row pass already flagged out-of-range values
         svd_row_info r;
         r.draft_token = -1; r.target_argmax = -1; r.accepted = -1; r.sample_token = -1;
@@ -1233,6 +1236,16 @@ __global__ void __launch_bounds__(256) finalize_kernel(const RowParams p) {
             if (lane == 0) {
                 p.accept_len[b] = a;
                 p.n_emitted[b] = a + (fix_row >= 0 ? 1 : 0);
+                // length-head labels: the observable proxy a / b_k and, verifying all k, a / k
+                if (p.bk_const > 0) {
+                    int nt = __ldg(p.bk_trunc + b);
+                    nt = nt < 1 ? 1 : (nt > k ? k : nt);
+                    if (p.label_proxy) p.label_proxy[b] = static_cast<float>(min(a, nt)) / static_cast<float>(nt);
+                    if (p.label_full) p.label_full[b] = static_cast<float>(a) / static_cast<float>(k);
+                } else {
+                    if (p.label_proxy) p.label_proxy[b] = static_cast<float>(a) / static_cast<float>(n);
+                    if (p.label_full) p.label_full[b] = kQNaN;
+                }
             }
         }
         if (distill) {
