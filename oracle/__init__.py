@@ -14,6 +14,8 @@ Which pins hold each function (see ``tests/test_oracle_*.py``):
   * ``distill``      -- KL = 0 when draft == target; RKL >= 0; K_c <= RKL; c = inf equals torch
                         kl_div; lambda = 1 equals torch cross_entropy; a hand-derived V = 2
                         golden case; finite differences; torch autograd; sum of gradient = 0.
+  * ``length_head_update`` -- torch fp64 autograd of an independent expression of the loss;
+                        a hand-derived one-unit case; three AdamW steps against torch.optim.AdamW.
   * ``speedup_report`` -- hand-counted small cases; all-accepted and all-rejected limits; the
                         closed form recovered from geometric accept lengths (i.i.d. rate A).
   * ``philox``       -- parity unpinned against published known-answer vectors (none are
@@ -61,6 +63,10 @@ def _load():
     lib.orc_length_head.restype = i32
     lib.orc_row_stats.argtypes = [P, i32, f64, P, P, P]
     lib.orc_speedup_report.argtypes = [P, P, P, i32, i32, f64, P]
+    lib.orc_length_head_update.argtypes = [P, P, i32, i32, i32, P, P, P, f64, P, P, P, P,
+                                           P, P, P, P, P, P, P, P, i32, f64, f64, f64, f64, f64,
+                                           P, P, P, P, P, P]
+    lib.orc_length_head_update.restype = i32
     lib.orc_speedup_report.restype = i32
     lib.orc_verify.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, f64, u64, u64,
                                P, P, P, P, P, P, P, P, P]
@@ -221,6 +227,42 @@ def distill(D, T, bk, lam: float, clip_c: float, tau: float = 1.0, grad_scale: f
 
 def expected_tokens(A: float, k: int) -> float:
     return float(_load().orc_expected_tokens(float(A), int(k)))
+
+
+def length_head_update(h, label, W1, b1, w2, b2: float, state: dict, step: int,
+                       lr: float = 2e-4, beta1: float = 0.9, beta2: float = 0.999,
+                       eps: float = 1e-8, wd: float = 0.01) -> dict:
+    """One AdamW step of the length head on l = mean_b (bhat_b - label_b)^2.
+
+    h, W1, w2: bf16 (the served forward weights); b1: fp32/fp64 [M]; b2: float.  ``state``
+    holds fp64 numpy arrays W1m, b1m, w2m, b2m (masters) and mW1, vW1, mb1, vb1, mw2, vw2,
+    mb2, vb2 (AdamW moments); they are updated in place.  Returns loss, bhat and the gradients.
+    """
+    hb, Wb, wb = _bits(h), _bits(W1), _bits(w2)
+    B, H = hb.shape
+    M = Wb.shape[0]
+    lab = np.ascontiguousarray(np.asarray(label, np.float64))
+    b1a = np.ascontiguousarray(np.asarray(b1, np.float64))
+    for key in ("W1m", "b1m", "w2m", "b2m", "mW1", "vW1", "mb1", "vb1", "mw2", "vw2", "mb2", "vb2"):
+        arr = state[key]
+        assert arr.dtype == np.float64 and arr.flags["C_CONTIGUOUS"], key
+    loss = np.zeros(1, np.float64)
+    bhat = np.zeros(B, np.float64)
+    gW1 = np.zeros((M, H), np.float64)
+    gb1 = np.zeros(M, np.float64)
+    gw2 = np.zeros(M, np.float64)
+    gb2 = np.zeros(1, np.float64)
+    S = state
+    rc = _load().orc_length_head_update(
+        _ptr(hb), _ptr(lab), B, H, M, _ptr(Wb), _ptr(b1a), _ptr(wb), float(b2),
+        _ptr(S["W1m"]), _ptr(S["b1m"]), _ptr(S["w2m"]), _ptr(S["b2m"]),
+        _ptr(S["mW1"]), _ptr(S["vW1"]), _ptr(S["mb1"]), _ptr(S["vb1"]),
+        _ptr(S["mw2"]), _ptr(S["vw2"]), _ptr(S["mb2"]), _ptr(S["vb2"]),
+        int(step), float(lr), float(beta1), float(beta2), float(eps), float(wd),
+        _ptr(loss), _ptr(bhat), _ptr(gW1), _ptr(gb1), _ptr(gw2), _ptr(gb2))
+    if rc != 0:
+        raise ValueError("oracle length_head_update: bad arguments")
+    return dict(loss=float(loss[0]), bhat=bhat, gW1=gW1, gb1=gb1, gw2=gw2, gb2=float(gb2[0]))
 
 
 def speedup_report(accept_len, bk, n_emitted, k: int, rho: float) -> np.ndarray:

@@ -543,3 +543,91 @@ int orc_speedup_report(const int32_t* accept_len, const int32_t* bk, const int32
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Length-head online update ([VR] load_bearing_attack: l_len = (bhat - a*)^2 trains the head  */
+/* online; [PR] Axiom ledger: length head learning rate 2e-4, AdamW).                          */
+/* Readings: the batch loss is the mean over sequences,                                        */
+/*   l = (1/B) sum_b (bhat_b - a*_b)^2;                                                          */
+/* the forward uses the bf16 weights as served (W1, w2) with fp32 biases; the gradient is      */
+/* applied to fp64 master weights (W1m, b1m, w2m, b2m) by one AdamW step (Loshchilov & Hutter, */
+/* "Decoupled Weight Decay Regularization", ICLR 2019; in the order torch.optim.AdamW uses:    */
+/* decay theta *= 1 - lr*wd, then m, v, bias corrections 1 - beta^t, theta -= lr*mhat/(sqrt(   */
+/* vhat) + eps)); no gradient flows into h.  ReLU'(0) = 0.                                      */
+/*   delta_b  = (2/B) (bhat_b - a*_b) bhat_b (1 - bhat_b)        (dl/dz_b)                      */
+/*   g_b2     = sum_b delta_b;       g_w2[m] = sum_b delta_b relu(a_bm)                         */
+/*   e_bm     = delta_b w2[m] [a_bm > 0];  g_b1[m] = sum_b e_bm;  g_W1[m,j] = sum_b e_bm h_bj    */
+/* ------------------------------------------------------------------------------------------ */
+static void adamw_step(double* theta, double* m, double* v, const double* g, size_t n, int t,
+                       double lr, double beta1, double beta2, double eps, double wd) {
+    const double bc1 = 1.0 - pow(beta1, (double)t), bc2 = 1.0 - pow(beta2, (double)t);
+    for (size_t i = 0; i < n; ++i) {
+        theta[i] *= 1.0 - lr * wd;
+        m[i] = beta1 * m[i] + (1.0 - beta1) * g[i];
+        v[i] = beta2 * v[i] + (1.0 - beta2) * g[i] * g[i];
+        const double mhat = m[i] / bc1, vhat = v[i] / bc2;
+        theta[i] -= lr * mhat / (sqrt(vhat) + eps);
+    }
+}
+
+int orc_length_head_update(const uint16_t* h, const double* label, int B, int H, int M,
+                           const uint16_t* W1, const double* b1, const uint16_t* w2, double b2,
+                           double* W1m, double* b1m, double* w2m, double* b2m,
+                           double* mW1, double* vW1, double* mb1, double* vb1,
+                           double* mw2, double* vw2, double* mb2, double* vb2,
+                           int step, double lr, double beta1, double beta2, double eps, double wd,
+                           double* loss_out, double* bhat_out,
+                           double* gW1, double* gb1, double* gw2, double* gb2 /* out */) {
+    if (B < 1 || H < 1 || M < 1 || step < 1) return 1;
+    double* a = (double*)malloc(sizeof(double) * (size_t)B * M);
+    double* delta = (double*)malloc(sizeof(double) * (size_t)B);
+    if (!a || !delta) { free(a); free(delta); return 2; }
+    /* forward with the served weights */
+    double loss = 0.0;
+    for (int b = 0; b < B; ++b) {
+        double z = b2;
+        for (int m = 0; m < M; ++m) {
+            double s = b1[m];
+            for (int j = 0; j < H; ++j)
+                s += bf16_to_f64(W1[(size_t)m * H + j]) * bf16_to_f64(h[(size_t)b * H + j]);
+            a[(size_t)b * M + m] = s;
+            z += bf16_to_f64(w2[m]) * (s > 0.0 ? s : 0.0);
+        }
+        const double bh = 1.0 / (1.0 + exp(-z));
+        bhat_out[b] = bh;
+        loss += (bh - label[b]) * (bh - label[b]);
+        delta[b] = (2.0 / (double)B) * (bh - label[b]) * bh * (1.0 - bh);
+    }
+    *loss_out = loss / (double)B;
+    /* backward */
+    double g2 = 0.0;
+    for (int b = 0; b < B; ++b) g2 += delta[b];
+    *gb2 = g2;
+    for (int m = 0; m < M; ++m) {
+        double sw = 0.0, sb = 0.0;
+        const double w2m_f = bf16_to_f64(w2[m]);
+        for (int b = 0; b < B; ++b) {
+            const double s = a[(size_t)b * M + m];
+            sw += delta[b] * (s > 0.0 ? s : 0.0);
+            sb += (s > 0.0) ? delta[b] * w2m_f : 0.0;
+        }
+        gw2[m] = sw;
+        gb1[m] = sb;
+        for (int j = 0; j < H; ++j) {
+            double g = 0.0;
+            for (int b = 0; b < B; ++b) {
+                const double s = a[(size_t)b * M + m];
+                if (s > 0.0) g += delta[b] * w2m_f * bf16_to_f64(h[(size_t)b * H + j]);
+            }
+            gW1[(size_t)m * H + j] = g;
+        }
+    }
+    /* AdamW on every parameter */
+    adamw_step(W1m, mW1, vW1, gW1, (size_t)M * H, step, lr, beta1, beta2, eps, wd);
+    adamw_step(b1m, mb1, vb1, gb1, (size_t)M, step, lr, beta1, beta2, eps, wd);
+    adamw_step(w2m, mw2, vw2, gw2, (size_t)M, step, lr, beta1, beta2, eps, wd);
+    adamw_step(b2m, mb2, vb2, gb2, 1, step, lr, beta1, beta2, eps, wd);
+    free(a);
+    free(delta);
+    return 0;
+}
