@@ -339,6 +339,22 @@ def main():
     red = parallel.reduce_metrics(ms_per_step, verified, accepted, emitted, loss, device=dev)
     value = red["verified"] / (red["ms"] / 1000.0)
 
+    # ---------------------------------------------------------------- length-head online update
+    trainer = api.LengthHeadTrainer(d["W1"], d["b1"], d["w2"], d["b2"], w.B)
+    label = (fused.accept_len.float() / bk.float()).contiguous()   # the proxy label a / b_k
+    for _ in range(3):
+        trainer.step(d["h"], label)
+    torch.cuda.synchronize()
+    u0 = torch.cuda.Event(enable_timing=True)
+    u1 = torch.cuda.Event(enable_timing=True)
+    n_upd = 50
+    u0.record(stream)
+    for _ in range(n_upd):
+        trainer.step(d["h"], label)
+    u1.record(stream)
+    torch.cuda.synchronize()
+    update_ms = u0.elapsed_time(u1) / n_upd
+
     # ---------------------------------------------------------------- roofline of the row pass
     rows_avg_ms = statistics.mean(rows_ms)
     alg = algorithmic_bytes(bk_host, w.k, w.kt, w.V)
@@ -411,6 +427,7 @@ def main():
             "emitted_tokens_per_s": red["emitted"] / (red["ms"] / 1000.0),
             "step_hbm_gbs": (alg + head_bytes(w.B, w.H, w.M)) * info.world / (red["ms"] / 1000.0) / 1e9,
             "length_head_avg_ms": statistics.mean(head_ms),
+            "length_head_update_ms": update_ms,
             "bk_hist": bk_hist,
             "speedup_report": {k_: (None if v_ != v_ else round(v_, 6)) for k_, v_ in report.items()
                                if k_ != "alpha"},

@@ -55,6 +55,18 @@ class VerifyDistillArgs(ctypes.Structure):
     ]
 
 
+class HeadUpdateArgs(ctypes.Structure):
+    """Mirror of ``svd_head_update_args``."""
+    _fields_ = [
+        ("h", _P), ("label", _P), ("B", _I), ("H", _I), ("M", _I),
+        ("W1m", _P), ("b1", _P), ("w2m", _P), ("b2", _P), ("W1", _P), ("w2", _P),
+        ("mW1", _P), ("vW1", _P), ("mb1", _P), ("vb1", _P), ("mw2", _P), ("vw2", _P),
+        ("mb2", _P), ("vb2", _P), ("step", _I),
+        ("lr", _F), ("beta1", _F), ("beta2", _F), ("eps", _F), ("weight_decay", _F),
+        ("loss", _P), ("bhat", _P),
+    ]
+
+
 _lib = None
 
 
@@ -82,9 +94,10 @@ def lib():
     L.svd_selftest_wait_timeout.argtypes = [_P, _SZ, _U64, _P]
     L.svd_verify_distill_noalloc.argtypes = [ctypes.POINTER(VerifyDistillArgs), _P, _P]
     L.svd_speedup_report.argtypes = [_P, _P, _P, _I, _I, ctypes.c_double, _P, _P]
+    L.svd_length_head_update.argtypes = [ctypes.POINTER(HeadUpdateArgs), _P, _SZ, _P]
     for fn in ("svd_workspace_reset", "svd_length_head", "svd_verify", "svd_distill_loss_grad",
                "svd_verify_distill", "svd_get_device_error", "svd_selftest_wait_timeout",
-               "svd_verify_distill_noalloc", "svd_speedup_report"):
+               "svd_verify_distill_noalloc", "svd_speedup_report", "svd_length_head_update"):
         getattr(L, fn).restype = _I
     _lib = L
     return L
@@ -296,6 +309,58 @@ class VerifyDistill:
 def svd_verify_distill(D, T, **kw) -> dict:
     """a1-a5 in one call; keyword arguments as in :class:`VerifyDistill`."""
     return VerifyDistill(D, T, **kw)().outputs()
+
+
+class LengthHeadTrainer:
+    """Online AdamW training of the length head through ``svd_length_head_update``.
+
+    Holds fp32 master weights, AdamW moments and the bf16 copies the forward serves
+    (``W1``, ``w2``; pass ``head()`` to :class:`VerifyDistill`).  Defaults: learning rate 2e-4
+    (the pages' value), betas (0.9, 0.999), eps 1e-8, weight decay 0.01.
+    """
+
+    def __init__(self, W1, b1, w2, b2: float, B: int, lr=2e-4, betas=(0.9, 0.999), eps=1e-8,
+                 weight_decay=0.01):
+        dev = W1.device
+        M, H = W1.shape
+        self.B, self.H, self.M = B, H, M
+        self.W1m = W1.float().contiguous().clone()
+        self.b1 = (torch.zeros(M, device=dev) if b1 is None else b1.float().clone()).contiguous()
+        self.w2m = w2.float().contiguous().clone()
+        self.b2 = torch.full((1,), float(b2), dtype=torch.float32, device=dev)
+        self.W1 = self.W1m.to(torch.bfloat16).contiguous()
+        self.w2 = self.w2m.to(torch.bfloat16).contiguous()
+        self.moments = [torch.zeros_like(t) for t in (self.W1m, self.W1m, self.b1, self.b1,
+                                                      self.w2m, self.w2m, self.b2, self.b2)]
+        self.loss = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.bhat = torch.zeros(B, dtype=torch.float32, device=dev)
+        self.ws = Workspace(B, 1, 1, M, device=dev)
+        self.step_count = 0
+        self.hyper = (float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay))
+
+    def head(self, h):
+        """The (h, W1, b1, w2, b2) tuple for :class:`VerifyDistill` (b2 read back from device)."""
+        return (h, self.W1, self.b1, self.w2, float(self.b2.item()))
+
+    def step(self, h, label, stream=None):
+        """One AdamW step on l = mean_b (bhat_b - label_b)^2; returns (loss, bhat) tensors."""
+        if h.shape != (self.B, self.H):
+            raise ValueError("h must be [B, H] = [%d, %d]" % (self.B, self.H))
+        self.step_count += 1
+        a = HeadUpdateArgs()
+        lab = label.float().contiguous()
+        self._label = lab   # alive until the launch is enqueued
+        a.h, a.label = _ptr(_bits(h)), _ptr(lab)
+        a.B, a.H, a.M = self.B, self.H, self.M
+        a.W1m, a.b1, a.w2m, a.b2 = _ptr(self.W1m), _ptr(self.b1), _ptr(self.w2m), _ptr(self.b2)
+        a.W1, a.w2 = _ptr(self.W1), _ptr(self.w2)
+        (a.mW1, a.vW1, a.mb1, a.vb1, a.mw2, a.vw2, a.mb2, a.vb2) = [_ptr(t) for t in self.moments]
+        a.step = self.step_count
+        a.lr, a.beta1, a.beta2, a.eps, a.weight_decay = self.hyper
+        a.loss, a.bhat = _ptr(self.loss), _ptr(self.bhat)
+        _check(lib().svd_length_head_update(ctypes.byref(a), self.ws.ptr, self.ws.nbytes,
+                                            _stream(stream)), "svd_length_head_update")
+        return self.loss, self.bhat
 
 
 REPORT_FIELDS = ("tau_measured", "acc", "tau_model", "eta_model", "eta_measured", "mean_bk",

@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_kernel(const HeadPara
             for (int z = 0; z < static_cast<int>(gridDim.z); ++z)
                 a += __ldcg(p.part + (static_cast<size_t>(z) * p.B + b) * p.M + m);
             if (p.b1) a += __ldg(p.b1 + m);
+            if (p.u_out) p.u_out[static_cast<size_t>(b) * p.M + m] = a;
             const float w2 = __uint_as_float(static_cast<uint32_t>(__ldg(p.w2 + m)) << 16);
             a = w2 * fmaxf(a, 0.f);
         }
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_kernel(const HeadPara
     __threadfence();
     const int mtiles = gridDim.y;
     for (int b = t; b < p.B; b += blockDim.x) {
-        float z = p.b2;
+        float z = p.b2_dev ? *p.b2_dev : p.b2;
         for (int q = 0; q < mtiles; ++q) z += __ldcg(p.zpart + static_cast<size_t>(q) * p.B + b);
         const float bhat = 1.f / (1.f + expf(-z));
         const float target = p.gamma * bhat * static_cast<float>(p.k);
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_kernel(const HeadPara
         int bk = static_cast<int>(fminf(fmaxf(r, 1.f), static_cast<float>(p.k)));
         if (!(r == r)) bk = 1;  // non-finite hidden states
         if (p.bhat) p.bhat[b] = bhat;
-        p.bk[b] = bk;
+        if (p.bk) p.bk[b] = bk;
     }
     if (t == 0) p.hdr->head_ticket = 0u;
 }

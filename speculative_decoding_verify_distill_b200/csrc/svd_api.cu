@@ -65,7 +65,7 @@ svd_status run_head(const uint16_t* h, const uint16_t* W1, const float* b1, cons
     p.h = h; p.W1 = W1; p.b1 = b1; p.w2 = w2; p.b2 = b2;
     p.B = B; p.H = H; p.M = M; p.k = k;
     p.gamma = gamma; p.rnd = static_cast<int>(rnd);
-    p.bhat = bhat_out; p.bk = bk_out;
+    p.bhat = bhat_out; p.bk = bk_out; p.b2_dev = nullptr; p.u_out = nullptr;
     p.hdr = w.hdr; p.zpart = w.zpart; p.part = w.part; p.tile_ticket = w.tile_ticket;
     p.nsplit = head_nsplit(B, M);
     const int per = (H + p.nsplit - 1) / p.nsplit;
@@ -222,6 +222,50 @@ svd_status svd_verify_distill(const svd_verify_distill_args* a, void* ws, size_t
                     a->dlogits, a->loss_rows, a->loss_total, a->accept_len, a->emitted,
                     a->n_emitted, a->row_info, w, stream, a->full_k ? a->k : 0, a->label_proxy,
                     a->label_full);
+}
+
+svd_status svd_length_head_update(const svd_head_update_args* a, void* ws, size_t ws_bytes,
+                                  void* stream) {
+    if (!a) return SVD_ERR_INVALID_ARG;
+    if (a->B < 1 || a->H < 1 || a->M < 1 || a->step < 1) return SVD_ERR_INVALID_ARG;
+    if (!a->h || !a->label || !a->W1m || !a->b1 || !a->w2m || !a->b2 || !a->W1 || !a->w2 ||
+        !a->mW1 || !a->vW1 || !a->mb1 || !a->vb1 || !a->mw2 || !a->vw2 || !a->mb2 || !a->vb2 ||
+        !a->loss || !a->bhat)
+        return SVD_ERR_INVALID_ARG;
+    if (bad_float(a->lr) || a->lr < 0.f || bad_float(a->weight_decay) || a->weight_decay < 0.f ||
+        !(a->beta1 >= 0.f && a->beta1 < 1.f) || !(a->beta2 >= 0.f && a->beta2 < 1.f) ||
+        bad_float(a->eps) || !(a->eps > 0.f))
+        return SVD_ERR_INVALID_ARG;
+    svd_status s = check_ws(ws, ws_bytes, a->B, 1, 1, a->M);
+    if (s != SVD_OK) return s;
+    const WsLayout L = ws_layout(a->B, 1, 1, a->M);
+    const WsPtrs w = carve(ws, a->B, 1, 1, a->M);
+    char* base = static_cast<char*>(ws);
+    float* u = reinterpret_cast<float*>(base + L.u);
+    float* e = reinterpret_cast<float*>(base + L.e);
+    // forward on the served weights, keeping the pre-activations
+    HeadParams hp;
+    hp.h = a->h; hp.W1 = a->W1; hp.b1 = a->b1; hp.w2 = a->w2; hp.b2 = 0.f;
+    hp.B = a->B; hp.H = a->H; hp.M = a->M; hp.k = 1;
+    hp.gamma = 1.f; hp.rnd = 0;
+    hp.bhat = a->bhat; hp.bk = nullptr; hp.b2_dev = a->b2; hp.u_out = u;
+    hp.hdr = w.hdr; hp.zpart = w.zpart; hp.part = w.part; hp.tile_ticket = w.tile_ticket;
+    hp.nsplit = head_nsplit(a->B, a->M);
+    const int per = (a->H + hp.nsplit - 1) / hp.nsplit;
+    hp.ks = (per + 15) & ~15;
+    s = from_cuda(launch_length_head(hp, stream));
+    if (s != SVD_OK) return s;
+    HeadUpdateParams p;
+    p.h = a->h; p.label = a->label; p.bhat = a->bhat; p.u = u; p.e = e;
+    p.B = a->B; p.H = a->H; p.M = a->M;
+    p.W1m = a->W1m; p.b1 = a->b1; p.w2m = a->w2m; p.b2 = a->b2; p.W1 = a->W1; p.w2 = a->w2;
+    p.mW1 = a->mW1; p.vW1 = a->vW1; p.mb1 = a->mb1; p.vb1 = a->vb1;
+    p.mw2 = a->mw2; p.vw2 = a->vw2; p.mb2 = a->mb2; p.vb2 = a->vb2;
+    p.lr = a->lr; p.beta1 = a->beta1; p.beta2 = a->beta2; p.eps = a->eps; p.wd = a->weight_decay;
+    p.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(a->beta1), a->step));
+    p.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(a->beta2), a->step));
+    p.loss = a->loss;
+    return from_cuda(launch_head_update(p, stream));
 }
 
 svd_status svd_speedup_report(const int32_t* accept_len, const int32_t* bk,

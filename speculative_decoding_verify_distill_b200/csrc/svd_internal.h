@@ -37,7 +37,7 @@ __host__ __device__ inline int head_nsplit(int B, int M) {
 }
 
 struct WsLayout {
-    size_t rec, seq_loss, zpart, part, tile_ticket, total;
+    size_t rec, seq_loss, zpart, part, tile_ticket, u, e, total;
 };
 
 __host__ __device__ inline WsLayout ws_layout(int B, int k, int kt, int M) {
@@ -56,6 +56,12 @@ __host__ __device__ inline WsLayout ws_layout(int B, int k, int kt, int M) {
     off = align256(off + sizeof(float) * (size_t)head_nsplit(B, M) * (size_t)B * (size_t)(M > 0 ? M : 0));
     L.tile_ticket = off;
     off = align256(off + sizeof(uint32_t) * (size_t)bt * (size_t)mt);
+    // length-head update: pre-activations W1 h + b1 and backward terms, [B, M] fp32 each
+    const size_t bm = (size_t)B * (size_t)(M > 0 ? M : 0);
+    L.u = off;
+    off = align256(off + sizeof(float) * bm);
+    L.e = off;
+    off = align256(off + sizeof(float) * bm);
     L.total = off;
     return L;
 }
@@ -73,7 +79,9 @@ struct HeadParams {
     float gamma;
     int rnd;
     float* bhat;
-    int32_t* bk;
+    int32_t* bk;             // or null (no verification length wanted)
+    const float* b2_dev;     // or null: b2 from device memory instead of the scalar
+    float* u_out;            // or null: [B, M] pre-activations W1 h + b1
     WsHeader* hdr;
     float* zpart;            // [ceil(M/64), B] per-tile logits
     float* part;             // [nsplit, B, M] split partials of W1 h
@@ -124,6 +132,20 @@ struct RowParams {
 int launch_length_head(const HeadParams& p, void* stream);
 int launch_row_pass(const RowParams& p, void* stream);
 int launch_wait_timeout_selftest(WsHeader* hdr, uint64_t limit_ns, void* stream);
+struct HeadUpdateParams {
+    const uint16_t* h;
+    const float* label;
+    const float* bhat;
+    const float* u;          // [B, M] pre-activations of the forward
+    float* e;                // [B, M] dl/d(pre-activation)
+    int B, H, M;
+    float *W1m, *b1, *w2m, *b2;
+    uint16_t *W1, *w2;
+    float *mW1, *vW1, *mb1, *vb1, *mw2, *vw2, *mb2, *vb2;
+    float lr, beta1, beta2, eps, wd, bc1, bc2;   // bc = 1 - beta^step
+    float* loss;
+};
+int launch_head_update(const HeadUpdateParams& p, void* stream);
 int launch_speedup_report(const int32_t* accept_len, const int32_t* bk, const int32_t* n_emitted,
                           int B, int k, double rho, double* out, void* stream);
 
