@@ -628,14 +628,12 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         // main pass: exp relative to the thread maxima (no rescaling) and the reverse-KL moment;
         // straight-line over all rounds (sentinel vectors contribute exact zeros).  A thread
         // holding sentinels only keeps a zero reference.
-        float emax[NV];
         float2 aD = make_float2(0.f, 0.f), aDd = make_float2(0.f, 0.f), aT = make_float2(0.f, 0.f);
         float dmax = kNegInf;
         const float AD = RD > -1e38f ? __fmul_rn(RD, k2) : 0.f, AT = RT > -1e38f ? __fmul_rn(RT, k2) : 0.f;
         const float2 K2 = make_float2(k2, k2);
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
-            emax[j] = 0.f;
             if (!need_lse) continue;
             const int lv = j * 32 + lane;
             float2 xt[4], et[4];
@@ -667,8 +665,6 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 if (DISTILL) {
                     dmax = fmaxf(dmax, fmaxf(fmaxf(fmaxf(dd[0].x, dd[0].y), fmaxf(dd[1].x, dd[1].y)),
                                              fmaxf(fmaxf(dd[2].x, dd[2].y), fmaxf(dd[3].x, dd[3].y))));
-                    emax[j] = fmaxf(fmaxf(fmaxf(ed[0].x, ed[0].y), fmaxf(ed[1].x, ed[1].y)),
-                                    fmaxf(fmaxf(ed[2].x, ed[2].y), fmaxf(ed[3].x, ed[3].y)));
                 }
             }
         }
@@ -813,10 +809,11 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         float clip_d = 0.f, clip_q = 0.f, n_clip = 0.f;
         uint32_t clipmask = 0;
         if (do_clip) {
-            const float fD = fast_exp2(AD - L2D);          // q = e * fD for this thread's exps
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
-                if (emax[j] * fD > qthr) {
+                // largest q of the vector, from its largest draft logit (exact bf16 max)
+                const float qv = fast_exp2(__fsub_rn(__fmul_rn(max8_bf16(myD[j * 32 + lane]), k2), L2D));
+                if (qv > qthr) {
                     clipmask |= 1u << j;
                     float xd[8], xt[8];
                     unpack8(myD[j * 32 + lane], xd);
@@ -1046,13 +1043,12 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 if (vi / vpw == warp) {
                     const int lvy = vi - wv0;
                     if ((lvy & 31) == lane) {
-                        float xd[8], xt[8];
-                        unpack8(myD[lvy], xd);
-                        unpack8(myT[lvy], xt);
-                        float dy = xd[0], ty = xt[0];
-#pragma unroll
-                        for (int q = 1; q < 8; ++q)
-                            if (q == (yl & 7)) { dy = xd[q]; ty = xt[q]; }
+                        // the two bf16 values straight from the staged vectors (dynamic index
+                        // into shared memory, not into a register array)
+                        const float dy = __uint_as_float(static_cast<uint32_t>(
+                            reinterpret_cast<const uint16_t*>(myD + lvy)[yl & 7]) << 16);
+                        const float ty = __uint_as_float(static_cast<uint32_t>(
+                            reinterpret_cast<const uint16_t*>(myT + lvy)[yl & 7]) << 16);
                         const float qa = fast_exp2(fmaf(dy, k2, -L2D));
                         float gy = qa * fmaf(Q, dy - ty, P);
                         if (do_clip) {
