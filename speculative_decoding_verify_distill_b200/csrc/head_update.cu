@@ -9,9 +9,10 @@
 // torch.optim.AdamW applies it: theta *= 1 - lr*wd, then the bias-corrected moment step.
 //
 // Kernels (the forward, with its pre-activations stored, is the length-head kernel):
-//   back1: per sequence delta_b = (2/B)(bhat_b - a*_b) bhat_b (1 - bhat_b); per unit m the
-//          gradients of w2 and b1 (sums over b in order) and e_bm = delta_b w2_m [u_bm > 0];
-//          CTA 0 also forms the loss and the b2 gradient.  AdamW on w2, b1, b2.
+//   back1: per sequence delta_b = (2/B)(bhat_b - a*_b) bhat_b (1 - bhat_b), staged in shared
+//          memory by chunks; per unit m the gradients of w2 and b1 (sums over b in order) and
+//          e_bm = delta_b w2_m [u_bm > 0]; CTA 0 also forms the loss and the b2 gradient (fixed
+//          reduction order).  AdamW on w2, b1, b2.
 //   back2: dl/dW1 = E^T h ([M,B] x [B,H], 0.27 GFLOP at B=128, H=4096, M=256) on fp32 CUDA
 //          cores with shared-memory tiles, each output summed over b in order; AdamW on W1 in
 //          the epilogue.  Too small and too precision-sensitive (Adam's first step is
@@ -55,34 +56,61 @@ __device__ __forceinline__ float delta_of(const HeadUpdateParams& p, int b) {
 }
 
 __global__ void __launch_bounds__(kBack1Threads) head_back1_kernel(const HeadUpdateParams p) {
-    const int t = threadIdx.x;
-    if (blockIdx.x == 0 && t == 0) {
-        // loss and the b2 gradient, summed over b in order
-        float l = 0.f, g2 = 0.f;
-        for (int b = 0; b < p.B; ++b) {
-            const float r = __ldg(p.bhat + b) - __ldg(p.label + b);
-            l += r * r;
-            g2 += delta_of(p, b);
-        }
-        *p.loss = l / static_cast<float>(p.B);
-        float m = *p.mb2, v = *p.vb2;
-        *p.b2 = adamw(*p.b2, g2, m, v, p);
-        *p.mb2 = m;
-        *p.vb2 = v;
-    }
+    __shared__ float sdelta[kBack1Threads * 4];      // delta_b for a chunk of sequences
+    __shared__ float sred[2][kBack1Threads / 32];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int m = blockIdx.x * kBack1Threads + t;
-    if (m >= p.M) return;
-    const float w2 = bf16_to_f32(p.w2[m]);   // the forward's weight
-    float gw = 0.f, gb = 0.f;
-    for (int b = 0; b < p.B; ++b) {
-        const float d = delta_of(p, b);
-        const size_t o = static_cast<size_t>(b) * p.M + m;
-        const float u = p.u[o];
-        const float ev = u > 0.f ? d * w2 : 0.f;
-        gw += d * fmaxf(u, 0.f);
-        gb += ev;
-        p.e[o] = ev;
+    const bool live = m < p.M;
+    const float w2 = live ? bf16_to_f32(p.w2[m]) : 0.f;   // the forward's weight
+    float gw = 0.f, gb = 0.f, l = 0.f, g2 = 0.f;
+    constexpr int kChunk = kBack1Threads * 4;
+    for (int b0 = 0; b0 < p.B; b0 += kChunk) {
+        const int nb = min(kChunk, p.B - b0);
+        for (int r = t; r < nb; r += kBack1Threads) {
+            const int b = b0 + r;
+            const float d = delta_of(p, b);
+            sdelta[r] = d;
+            if (blockIdx.x == 0) {          // loss and b2 gradient: fixed per-thread strides
+                const float e = __ldg(p.bhat + b) - __ldg(p.label + b);
+                l += e * e;
+                g2 += d;
+            }
+        }
+        __syncthreads();
+        if (live) {
+#pragma unroll 4
+            for (int r = 0; r < nb; ++r) {   // sequences in order
+                const float d = sdelta[r];
+                const size_t o = static_cast<size_t>(b0 + r) * p.M + m;
+                const float u = p.u[o];
+                const float ev = u > 0.f ? d * w2 : 0.f;
+                gw += d * fmaxf(u, 0.f);
+                gb += ev;
+                p.e[o] = ev;
+            }
+        }
+        __syncthreads();
     }
+    if (blockIdx.x == 0) {
+        // fixed-order reduction of the per-thread partials: warp butterflies, then warps in order
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            l += __shfl_xor_sync(0xffffffffu, l, o);
+            g2 += __shfl_xor_sync(0xffffffffu, g2, o);
+        }
+        if (lane == 0) { sred[0][warp] = l; sred[1][warp] = g2; }
+        __syncthreads();
+        if (t == 0) {
+            float ls = 0.f, gs = 0.f;
+            for (int q = 0; q < kBack1Threads / 32; ++q) { ls += sred[0][q]; gs += sred[1][q]; }
+            *p.loss = ls / static_cast<float>(p.B);
+            float mm = *p.mb2, vv = *p.vb2;
+            *p.b2 = adamw(*p.b2, gs, mm, vv, p);
+            *p.mb2 = mm;
+            *p.vb2 = vv;
+        }
+    }
+    if (!live) return;
     float mm = p.mw2[m], vv = p.vw2[m];
     const float w2n = adamw(p.w2m[m], gw, mm, vv, p);
     p.w2m[m] = w2n;
