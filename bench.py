@@ -355,6 +355,26 @@ def main():
     torch.cuda.synchronize()
     update_ms = u0.elapsed_time(u1) / n_upd
 
+    # ---------------------------------------------------------------- full-k label mode
+    # the same step verifying and distilling all k rows (labels a/b_k and a/k both observable)
+    fullk = api.VerifyDistill(d["D"], d["T"], head=head, draft_tok=draft, mode=w.mode,
+                              temperature=w.tau, seed=w.philox_seed, lam=w.lam, clip_c=w.clip_c,
+                              ws=ws, full_k=True, labels=True)
+    for _ in range(3):
+        fullk()
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    n_fk = 20
+    f0.record(stream)
+    for _ in range(n_fk):
+        fullk()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fullk_ms = f0.elapsed_time(f1) / n_fk
+    fullk_bytes = algorithmic_bytes(np.full(w.B, w.k, np.int64), w.k, w.kt, w.V)
+    del fullk
+
     # ---------------------------------------------------------------- roofline of the row pass
     rows_avg_ms = statistics.mean(rows_ms)
     alg = algorithmic_bytes(bk_host, w.k, w.kt, w.V)
@@ -428,6 +448,8 @@ def main():
             "step_hbm_gbs": (alg + head_bytes(w.B, w.H, w.M)) * info.world / (red["ms"] / 1000.0) / 1e9,
             "length_head_avg_ms": statistics.mean(head_ms),
             "length_head_update_ms": update_ms,
+            "full_k_step_ms": fullk_ms,
+            "full_k_step_hbm_gbs": fullk_bytes / (fullk_ms / 1000.0) / 1e9,
             "bk_hist": bk_hist,
             "speedup_report": {k_: (None if v_ != v_ else round(v_, 6)) for k_, v_ in report.items()
                                if k_ != "alpha"},
