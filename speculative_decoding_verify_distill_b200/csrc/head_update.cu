@@ -10,9 +10,9 @@
 //
 // Kernels (the forward, with its pre-activations stored, is the length-head kernel):
 //   back1: per sequence delta_b = (2/B)(bhat_b - a*_b) bhat_b (1 - bhat_b), staged in shared
-//          memory by chunks; per unit m the gradients of w2 and b1 (sums over b in order) and
-//          e_bm = delta_b w2_m [u_bm > 0]; CTA 0 also forms the loss and the b2 gradient (fixed
-//          reduction order).  AdamW on w2, b1, b2.
+//          memory by chunks; per unit m the gradients of w2 and b1 and e_bm = delta_b w2_m
+//          [u_bm > 0] (32 units per CTA, 8 warps over the sequences, partials added in a fixed
+//          order); CTA 0 also forms the loss and the b2 gradient.  AdamW on w2, b1, b2.
 //   back2: dl/dW1 = E^T h ([M,B] x [B,H], 0.27 GFLOP at B=128, H=4096, M=256) on fp32 CUDA
 //          cores with shared-memory tiles, each output summed over b in order; AdamW on W1 in
 //          the epilogue.  Too small and too precision-sensitive (Adam's first step is
@@ -55,15 +55,19 @@ __device__ __forceinline__ float delta_of(const HeadUpdateParams& p, int b) {
     return (2.f / static_cast<float>(p.B)) * (bh - __ldg(p.label + b)) * bh * (1.f - bh);
 }
 
+// One CTA per 32 hidden units (lane = unit); its 8 warps take every 8th sequence, so each thread
+// walks B/8 sequences with independent loads, and the warps' partial sums are added in order.
 __global__ void __launch_bounds__(kBack1Threads) head_back1_kernel(const HeadUpdateParams p) {
-    __shared__ float sdelta[kBack1Threads * 4];      // delta_b for a chunk of sequences
-    __shared__ float sred[2][kBack1Threads / 32];
+    constexpr int kW = kBack1Threads / 32;
+    constexpr int kChunk = 1024;
+    __shared__ float sdelta[kChunk];                 // delta_b for a chunk of sequences
+    __shared__ float sred[2][kW][32];
+    __shared__ float sloss[2][kW];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int m = blockIdx.x * kBack1Threads + t;
+    const int m = blockIdx.x * 32 + lane;
     const bool live = m < p.M;
     const float w2 = live ? bf16_to_f32(p.w2[m]) : 0.f;   // the forward's weight
     float gw = 0.f, gb = 0.f, l = 0.f, g2 = 0.f;
-    constexpr int kChunk = kBack1Threads * 4;
     for (int b0 = 0; b0 < p.B; b0 += kChunk) {
         const int nb = min(kChunk, p.B - b0);
         for (int r = t; r < nb; r += kBack1Threads) {
@@ -78,8 +82,8 @@ __global__ void __launch_bounds__(kBack1Threads) head_back1_kernel(const HeadUpd
         }
         __syncthreads();
         if (live) {
-#pragma unroll 4
-            for (int r = 0; r < nb; ++r) {   // sequences in order
+#pragma unroll 8
+            for (int r = warp; r < nb; r += kW) {   // this warp's sequences, in order
                 const float d = sdelta[r];
                 const size_t o = static_cast<size_t>(b0 + r) * p.M + m;
                 const float u = p.u[o];
@@ -91,26 +95,31 @@ __global__ void __launch_bounds__(kBack1Threads) head_back1_kernel(const HeadUpd
         }
         __syncthreads();
     }
+    sred[0][warp][lane] = gw;
+    sred[1][warp][lane] = gb;
     if (blockIdx.x == 0) {
-        // fixed-order reduction of the per-thread partials: warp butterflies, then warps in order
+        // fixed-order reduction of the loss / b2 partials: warp butterflies, then warps in order
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             l += __shfl_xor_sync(0xffffffffu, l, o);
             g2 += __shfl_xor_sync(0xffffffffu, g2, o);
         }
-        if (lane == 0) { sred[0][warp] = l; sred[1][warp] = g2; }
-        __syncthreads();
-        if (t == 0) {
-            float ls = 0.f, gs = 0.f;
-            for (int q = 0; q < kBack1Threads / 32; ++q) { ls += sred[0][q]; gs += sred[1][q]; }
-            *p.loss = ls / static_cast<float>(p.B);
-            float mm = *p.mb2, vv = *p.vb2;
-            *p.b2 = adamw(*p.b2, gs, mm, vv, p);
-            *p.mb2 = mm;
-            *p.vb2 = vv;
-        }
+        if (lane == 0) { sloss[0][warp] = l; sloss[1][warp] = g2; }
     }
-    if (!live) return;
+    __syncthreads();
+    if (blockIdx.x == 0 && t == 0) {
+        float ls = 0.f, gs = 0.f;
+        for (int q = 0; q < kW; ++q) { ls += sloss[0][q]; gs += sloss[1][q]; }
+        *p.loss = ls / static_cast<float>(p.B);
+        float mm = *p.mb2, vv = *p.vb2;
+        *p.b2 = adamw(*p.b2, gs, mm, vv, p);
+        *p.mb2 = mm;
+        *p.vb2 = vv;
+    }
+    if (warp != 0 || !live) return;
+    gw = 0.f;
+    gb = 0.f;
+    for (int q = 0; q < kW; ++q) { gw += sred[0][q][lane]; gb += sred[1][q][lane]; }
     float mm = p.mw2[m], vv = p.vw2[m];
     const float w2n = adamw(p.w2m[m], gw, mm, vv, p);
     p.w2m[m] = w2n;
@@ -181,7 +190,7 @@ __global__ void __launch_bounds__(256) head_back2_kernel(const HeadUpdateParams 
 
 int launch_head_update(const HeadUpdateParams& p, void* stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    head_back1_kernel<<<(p.M + kBack1Threads - 1) / kBack1Threads, kBack1Threads, 0, st>>>(p);
+    head_back1_kernel<<<(p.M + 31) / 32, kBack1Threads, 0, st>>>(p);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return static_cast<int>(err);
     dim3 grid((p.H + kTile - 1) / kTile, (p.M + kTile - 1) / kTile);
