@@ -91,6 +91,24 @@ def test_block_sizes(k, kt):
     assert (vd.n_emitted.cpu().numpy() == (k + 1 if kt == k + 1 else k)).all()
 
 
+@pytest.mark.parametrize("B", [4096, 4097])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_batch_size_boundary_of_the_compact_lists(B, mode):
+    # up to 4096 sequences the row pass keeps b_k and the loaded / zero-row prefixes in shared
+    # memory and hands out work dynamically; above, it walks (sequence, row) slots in a fixed order
+    k, V = 3, 64
+    D, T = make_case(B, k, k + 1, V, seed=B + mode)
+    bk = syn.random_bk(B, k, B + 7)
+    draft = syn.sample_draft_tokens_batched(D, 1.0, B) if mode == 1 else None
+    vd = fused(D, T, bk, draft=draft, mode=mode, seed=11)
+    full_compare(vd, D, T, bk, draft=draft, mode=mode, seed=11)
+    g = vd.outputs()["dlogits"].cpu()
+    for b in range(0, B, 97):   # gradient rows past b_k are zero
+        n = int(bk[b])
+        if n < k:
+            assert int(torch.count_nonzero(g[b, n:])) == 0
+
+
 def test_argmax_ties_across_cluster_ranks():
     # V = 40960 runs as a cluster of two CTAs: ties are placed in both halves and in one vector
     B, k, V = 1, 4, 40960
