@@ -429,7 +429,7 @@ def main():
             "steps": K, "warmup": args.warmup, "ms_per_step": red["ms"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": args.workload, "B": w.B, "k": w.k, "kt": w.kt, "V": w.V, "H": w.H,
-                       "M": w.M, "mode": "greedy", "lambda": w.lam, "clip_c": w.clip_c,
+                       "M": w.M, "mode": "stochastic" if w.mode == 1 else "greedy", "lambda": w.lam, "clip_c": w.clip_c,
                        "storage": "bf16 logits / bf16 gradient, fp32 arithmetic",
                        "l2": "inputs larger than L2 (%.2f GB of logits per step, no flush)"
                              % ((host["D"].numel() + host["T"].numel()) * 2 / 1e9),
