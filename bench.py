@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 from speculative_decoding_verify_distill_b200 import api  # noqa: E402
 from speculative_decoding_verify_distill_b200 import parallel  # noqa: E402
 from speculative_decoding_verify_distill_b200 import synthetic as syn  # noqa: E402
+from speculative_decoding_verify_distill_b200 import vocab_parallel  # noqa: E402
 
 WORKLOAD = "ragged_qwen_b128"
 METRIC = "verified draft tokens/s and fused-pass HBM GB/s (% of B200 peak) at B=128,k=16"
@@ -224,6 +225,48 @@ def run_reference(args, info):
     print(json.dumps(line), flush=True)
 
 
+def time_vocab_shard(w, d, bk, bk_host, draft, P, stream, n=20):
+    """One rank's calls of the P-way vocab-sharded pass over this workload's rows (rank 0's
+    slice).  The other ranks' records come from one emulated step on this GPU; the two
+    all-gathers between the calls (NVLink, exchange_bytes_per_rank per rank) are not timed."""
+    slices = vocab_parallel.vocab_slices(w.V, P)
+    shards = [api.VocabShard(d["D"][..., v0:v0 + nv].contiguous(), d["T"][..., v0:v0 + nv].contiguous(),
+                             bk, V=w.V, v0=v0, P=P, rank=r, draft_tok=draft, mode=w.mode,
+                             temperature=w.tau, seed=w.philox_seed, lam=w.lam, clip_c=w.clip_c)
+              for r, (v0, nv) in enumerate(slices)]
+    vocab_parallel.run_emulated(shards, stream)
+    s0 = shards[0]
+    for _ in range(3):
+        s0.stats(stream)
+        s0.resolve(stream)
+        s0.finish(stream)
+    torch.cuda.synchronize()
+    if s0.device_error() != 0:
+        raise SystemExit("device error in the vocab-sharded pass")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    for j in range(n):
+        ev[j][0].record(stream)
+        s0.stats(stream)
+        ev[j][1].record(stream)
+        s0.resolve(stream)
+        ev[j][2].record(stream)
+        s0.finish(stream)
+        ev[j][3].record(stream)
+    torch.cuda.synchronize()
+    part = [statistics.mean(ev[j][q].elapsed_time(ev[j][q + 1]) for j in range(n)) for q in range(3)]
+    rank_ms = statistics.mean(ev[j][0].elapsed_time(ev[j][3]) for j in range(n))
+    Vl = slices[0][1]
+    alg = algorithmic_bytes(bk_host, w.k, w.kt, Vl)
+    n1 = api.svd_vs_exchange_bytes(w.B, w.kt, 1)
+    n2 = api.svd_vs_exchange_bytes(w.B, w.kt, 2)
+    del shards, s0
+    return {"P": P, "slice": Vl, "rank_step_ms": rank_ms, "stats_ms": part[0],
+            "resolve_ms": part[1], "finish_ms": part[2],
+            "rank_algorithmic_bytes": alg, "rank_hbm_gbs": alg / (rank_ms / 1000.0) / 1e9,
+            "exchange_bytes_per_rank": n1 + n2, "launches_per_rank_step": 5,
+            "note": "all-gathers not timed (one GPU)"}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -234,6 +277,7 @@ def main():
     ap.add_argument("--cpu-seqs", type=int, default=0, help="oracle sample size (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-vocab-shard", action="store_true", help="skip the vocab-sharded leg")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(syn.WORKLOADS),
                     help="profiling only: the reported bench line is the default workload")
     args = ap.parse_args()
@@ -375,6 +419,11 @@ def main():
     fullk_bytes = algorithmic_bytes(np.full(w.B, w.k, np.int64), w.k, w.kt, w.V)
     del fullk
 
+    # ---------------------------------------------------------------- vocab-sharded variant
+    vshard = None
+    if not args.no_vocab_shard and info.world == 1:
+        vshard = time_vocab_shard(w, d, bk, bk_host, draft, 8, stream)
+
     # ---------------------------------------------------------------- roofline of the row pass
     rows_avg_ms = statistics.mean(rows_ms)
     alg = algorithmic_bytes(bk_host, w.k, w.kt, w.V)
@@ -451,6 +500,7 @@ def main():
             "full_k_step_ms": fullk_ms,
             "full_k_step_hbm_gbs": fullk_bytes / (fullk_ms / 1000.0) / 1e9,
             "bk_hist": bk_hist,
+            "vocab_sharded": vshard,
             "speedup_report": {k_: (None if v_ != v_ else round(v_, 6)) for k_, v_ in report.items()
                                if k_ != "alpha"},
         }

@@ -67,6 +67,18 @@ class HeadUpdateArgs(ctypes.Structure):
     ]
 
 
+class VsArgs(ctypes.Structure):
+    """Mirror of ``svd_vs_args`` (include/svd_vocab.h)."""
+    _fields_ = [
+        ("D", _P), ("T", _P), ("draft_tok", _P), ("bk", _P), ("B", _I), ("k", _I), ("kt", _I),
+        ("V", _I), ("v0", _I), ("Vl", _I), ("P", _I), ("rank", _I), ("mode", _I),
+        ("temperature", _F), ("seed", _U64), ("step", _U64), ("distill", _I),
+        ("lambda_", _F), ("clip_c", _F), ("grad_scale", _F), ("dlogits", _P), ("dlogits_fp32", _I),
+        ("loss_rows", _P), ("loss_total", _P), ("accept_len", _P), ("emitted", _P),
+        ("n_emitted", _P), ("row_info", _P),
+    ]
+
+
 _lib = None
 
 
@@ -95,9 +107,17 @@ def lib():
     L.svd_verify_distill_noalloc.argtypes = [ctypes.POINTER(VerifyDistillArgs), _P, _P]
     L.svd_speedup_report.argtypes = [_P, _P, _P, _I, _I, ctypes.c_double, _P, _P]
     L.svd_length_head_update.argtypes = [ctypes.POINTER(HeadUpdateArgs), _P, _SZ, _P]
+    L.svd_vs_exchange_bytes.argtypes = [_I, _I, _I]
+    L.svd_vs_exchange_bytes.restype = _SZ
+    L.svd_vs_workspace_bytes.argtypes = [_I, _I, _I]
+    L.svd_vs_workspace_bytes.restype = _SZ
+    L.svd_vs_stats.argtypes = [ctypes.POINTER(VsArgs), _P, _P, _SZ, _P]
+    L.svd_vs_resolve.argtypes = [ctypes.POINTER(VsArgs), _P, _P, _P, _SZ, _P]
+    L.svd_vs_finish.argtypes = [ctypes.POINTER(VsArgs), _P, _P, _SZ, _P]
     for fn in ("svd_workspace_reset", "svd_length_head", "svd_verify", "svd_distill_loss_grad",
                "svd_verify_distill", "svd_get_device_error", "svd_selftest_wait_timeout",
-               "svd_verify_distill_noalloc", "svd_speedup_report", "svd_length_head_update"):
+               "svd_verify_distill_noalloc", "svd_speedup_report", "svd_length_head_update",
+               "svd_vs_stats", "svd_vs_resolve", "svd_vs_finish"):
         getattr(L, fn).restype = _I
     _lib = L
     return L
@@ -406,3 +426,102 @@ def svd_selftest_wait_timeout(ws: Workspace, limit_ns: int, stream=None) -> None
 
 
 INF = math.inf
+
+
+# ------------------------------------------------------------------------------------------
+# vocab-sharded pass (include/svd_vocab.h)
+# ------------------------------------------------------------------------------------------
+def svd_vs_exchange_bytes(B: int, kt: int, which: int) -> int:
+    return int(lib().svd_vs_exchange_bytes(B, kt, which))
+
+
+def svd_vs_workspace_bytes(B: int, k: int, kt: int) -> int:
+    return int(lib().svd_vs_workspace_bytes(B, k, kt))
+
+
+class VocabShard:
+    """One rank's part of the vocab-sharded verify-and-distill pass.
+
+    ``D`` [B, k, Vl] and ``T`` [B, kt, Vl] are this rank's slices (ids ``v0 .. v0+Vl-1``) of
+    the logit rows.  The three calls ``svd_vs_stats``, ``svd_vs_resolve`` and ``svd_vs_finish``
+    read and write the exchange buffers ``send1``/``recv1`` and ``send2``/``recv2`` (uint8,
+    rank r's records at block r of ``recv*``); moving ``send*`` of every rank into ``recv*``
+    is the caller's all-gather (``vocab_parallel``)."""
+
+    def __init__(self, D, T, bk, *, V: int, v0: int, P: int, rank: int, draft_tok=None,
+                 mode: int = GREEDY, temperature: float = 1.0, seed: int = 0, step: int = 0,
+                 distill: bool = True, lam: float = 0.5, clip_c: float = 1.0,
+                 grad_scale: float = 1.0, dlogits_fp32: bool = False, row_info: bool = False):
+        B, k, Vl = D.shape
+        kt = T.shape[1]
+        dev = D.device
+        self.shape = (B, k, kt, V, v0, Vl, P, rank)
+        self.mode = int(mode)
+        self.distill = bool(distill)
+        self._keep = [_bits(D), _bits(T), bk, draft_tok]
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.accept_len = torch.empty(B, **i32)
+        self.emitted = torch.empty((B, k + 1), **i32)
+        self.n_emitted = torch.empty(B, **i32)
+        self.loss_rows = torch.empty((B, k), dtype=torch.float32, device=dev) if distill else None
+        self.loss_total = torch.empty(1, dtype=torch.float32, device=dev) if distill else None
+        self.dlogits = (torch.empty((B, k, Vl), dtype=torch.float32 if dlogits_fp32 else torch.bfloat16,
+                                    device=dev) if distill else None)
+        self.row_info = _row_info_tensor(B, kt, dev) if row_info else None
+        u8 = dict(dtype=torch.uint8, device=dev)
+        n1, n2 = svd_vs_exchange_bytes(B, kt, 1), svd_vs_exchange_bytes(B, kt, 2)
+        self.send1 = torch.empty(max(n1, 16), **u8)
+        self.recv1 = torch.empty(max(P * n1, 16), **u8)
+        self.send2 = torch.empty(max(n2, 16), **u8)
+        self.recv2 = torch.empty(max(P * n2, 16), **u8)
+        nw = max(svd_vs_workspace_bytes(B, k, kt), 256)
+        self.ws = torch.zeros(nw, **u8)
+        assert self.ws.data_ptr() % 256 == 0
+        a = VsArgs()
+        a.D, a.T = _ptr(D), _ptr(T)
+        a.draft_tok, a.bk = _ptr(draft_tok), _ptr(bk)
+        a.B, a.k, a.kt, a.V, a.v0, a.Vl, a.P, a.rank = B, k, kt, V, v0, Vl, P, rank
+        a.mode, a.temperature, a.seed, a.step = int(mode), float(temperature), int(seed), int(step)
+        a.distill = 1 if distill else 0
+        a.lambda_, a.clip_c, a.grad_scale = float(lam), float(clip_c), float(grad_scale)
+        a.dlogits, a.dlogits_fp32 = _ptr(self.dlogits), 1 if dlogits_fp32 else 0
+        a.loss_rows, a.loss_total = _ptr(self.loss_rows), _ptr(self.loss_total)
+        a.accept_len, a.emitted, a.n_emitted = _ptr(self.accept_len), _ptr(self.emitted), _ptr(self.n_emitted)
+        a.row_info = _ptr(self.row_info)
+        self.args = a
+
+    @property
+    def stochastic(self) -> bool:
+        return self.mode == STOCHASTIC
+
+    def set_step(self, step: int):
+        self.args.step = int(step)
+
+    def _ws(self):
+        return ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel()
+
+    def stats(self, stream=None):
+        w, n = self._ws()
+        _check(lib().svd_vs_stats(ctypes.byref(self.args), _ptr(self.send1), w, n, _stream(stream)),
+               "svd_vs_stats")
+
+    def resolve(self, stream=None):
+        w, n = self._ws()
+        _check(lib().svd_vs_resolve(ctypes.byref(self.args), _ptr(self.recv1), _ptr(self.send2), w, n,
+                                    _stream(stream)), "svd_vs_resolve")
+
+    def finish(self, stream=None):
+        w, n = self._ws()
+        _check(lib().svd_vs_finish(ctypes.byref(self.args), _ptr(self.recv2), w, n, _stream(stream)),
+               "svd_vs_finish")
+
+    def device_error(self, stream=None) -> int:
+        return int(lib().svd_get_device_error(ctypes.c_void_p(self.ws.data_ptr()), _stream(stream)))
+
+    def outputs(self) -> dict:
+        out = dict(accept_len=self.accept_len, emitted=self.emitted, n_emitted=self.n_emitted)
+        if self.distill:
+            out.update(loss_rows=self.loss_rows, loss_total=self.loss_total, dlogits=self.dlogits)
+        if self.row_info is not None:
+            out["row_info"] = self.row_info
+        return out

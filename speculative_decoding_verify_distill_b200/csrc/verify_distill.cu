@@ -117,22 +117,6 @@ __device__ __forceinline__ Item unpack_item(uint32_t v) {
     if ((v & 3u) == 0u) return Item{kItemNone, -1, -1};
     return Item{static_cast<int>(v & 3u), static_cast<int>(v >> 8), static_cast<int>((v >> 2) & 63u)};
 }
-// Position (0..7) of the first element of a bf16 vector equal to R (7 if none: never used then).
-__device__ __forceinline__ int first_pos(const uint4& v, float R) {
-    float x[8];
-    unpack8(v, x);
-    int l = 7;
-#pragma unroll
-    for (int q = 6; q >= 0; --q) l = (x[q] == R) ? q : l;
-    return l;
-}
-// The four bf16 pairs of a 16-byte vector as packed fp32 pairs (exact).
-__device__ __forceinline__ void unpack8x2(const uint4& v, float2 (&x)[4]) {
-    x[0] = make_float2(bf_lo(v.x), bf_hi(v.x));
-    x[1] = make_float2(bf_lo(v.y), bf_hi(v.y));
-    x[2] = make_float2(bf_lo(v.z), bf_hi(v.z));
-    x[3] = make_float2(bf_lo(v.w), bf_hi(v.w));
-}
 __device__ __forceinline__ Msg1 empty_msg1() {
     Msg1 m;
     m.mD = m.mT = m.dmax = kNegInf;
@@ -211,56 +195,6 @@ __device__ __forceinline__ int loaded_slots(const RowParams& p, const int* spre)
     return spre ? spre[p.B] : p.B * p.kt;
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-// Factor that moves a sum taken relative to reference round(m k2) onto round(M k2) (exactly 1
-// when m == M).  Maxima at or below -1e38 mark empty sums (all -inf, or the staging sentinel).
-__device__ __forceinline__ float rescale(float m, float M, float k2) {
-    return m > -1e38f ? fast_exp2(__fsub_rn(__fmul_rn(m, k2), __fmul_rn(M, k2))) : 0.f;
-}
-
-// Per-element quantities with explicit rounding (no contraction), so that the values summed in
-// pass B and the values recomputed later (clip decisions, sample search) are bit-identical.
-// q_v = exp(D_v / tau - lseD) and p_v = exp(T_v / tau - lseT) from the staged bf16 logits.
-__device__ __forceinline__ float elem_q(float xd, float k2, float L2D) {
-    return fast_exp2(__fmaf_rn(xd, k2, -L2D));
-}
-__device__ __forceinline__ float elem_p(float xt, float k2, float L2T) {
-    return fast_exp2(__fmaf_rn(xt, k2, -L2T));
-}
-__device__ __forceinline__ float elem_s(float xd, float xt, float itau, float dl) {
-    return __fmaf_rn(__fsub_rn(xd, xt), itau, -dl);
-}
-__device__ __forceinline__ float elem_d(float q, float s) { return __fmul_rn(q, s); }
-// Sample masses as 2^-48 fixed-point integers: exact, associative prefix sums.
-__device__ __forceinline__ unsigned long long to_fixed(float r) {
-    return __float2ull_rz(r * 281474976710656.0f);
-}
-
-// floor(R * u24 / 2^24) exactly, for u24 < 2^24 and R < 2^63.
-__device__ __forceinline__ unsigned long long scale_mass(unsigned long long R, uint32_t u24) {
-    const unsigned long long lo = R * static_cast<unsigned long long>(u24);
-    const unsigned long long hi = __umul64hi(R, static_cast<unsigned long long>(u24));
-    return (lo >> 24) | (hi << 40);
-}
-
-
-__device__ __forceinline__ void warp_inclusive_scan_u64(unsigned long long& x) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-}
 
 }  // namespace
 

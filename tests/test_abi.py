@@ -13,6 +13,8 @@ from speculative_decoding_verify_distill_b200 import build as svd_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "svd.h")
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
 
 
 @pytest.fixture(scope="module")
@@ -22,7 +24,7 @@ def L():
 
 
 def declared_functions():
-    src = open(HEADER).read()
+    src = "\n".join(open(h).read() for h in HEADERS)
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(svd_[a-z_]+)\s*\(", src, flags=re.M)
     return sorted(set(names))
@@ -108,3 +110,73 @@ def test_fused_args_struct_matches_header():
     decls = [d.strip() for d in body.split("{", 1)[1].split(";") if d.strip()]
     n = sum(len(d.split(",")) for d in decls)
     assert n == len(api.VerifyDistillArgs._fields_)
+
+
+def test_vocab_header_declares_the_sharded_calls():
+    names = declared_functions()
+    for n in ("svd_vs_stats", "svd_vs_resolve", "svd_vs_finish", "svd_vs_exchange_bytes",
+              "svd_vs_workspace_bytes"):
+        assert n in names, n
+
+
+def _c_layout(struct, fields, tmp_path):
+    """sizeof and field offsets of a header struct, from a C program built with gcc."""
+    import subprocess
+    src = tmp_path / "layout.c"
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "svd_vocab.h"', "int main(void) {",
+             '  printf("%%zu\\n", sizeof(%s));' % struct]
+    for f in fields:
+        lines.append('  printf("%%zu\\n", offsetof(%s, %s));' % (struct, f))
+    lines.append("  return 0;\n}")
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    return int(out[0]), [int(x) for x in out[1:]]
+
+
+@pytest.mark.parametrize("struct,mirror", [("svd_vs_args", api.VsArgs),
+                                           ("svd_verify_distill_args", api.VerifyDistillArgs),
+                                           ("svd_head_update_args", api.HeadUpdateArgs)])
+def test_ctypes_mirrors_match_the_c_layout(struct, mirror, tmp_path):
+    names = [f[0] for f in mirror._fields_]
+    size, offs = _c_layout(struct, [("lambda" if n == "lambda_" else n) for n in names], tmp_path)
+    assert size == ctypes.sizeof(mirror)
+    assert offs == [getattr(mirror, n).offset for n in names]
+
+
+def test_vocab_sizes_and_argument_errors(L):
+    assert L.svd_vs_exchange_bytes(128, 17, 1) == 128 * 17 * 48
+    assert L.svd_vs_exchange_bytes(128, 17, 2) == 128 * 17 * 32
+    assert L.svd_vs_exchange_bytes(128, 17, 3) == 0
+    assert L.svd_vs_workspace_bytes(4, 8, 10) == 0
+    assert L.svd_vs_workspace_bytes(128, 16, 17) > 128 * 17 * 64
+    fake = ctypes.c_void_p(0x1000)   # never dereferenced: validation fails first
+    ws = ctypes.c_void_p(0x10000)
+
+    def args(**kw):
+        a = api.VsArgs()
+        a.D = a.T = a.bk = a.accept_len = a.emitted = a.n_emitted = a.dlogits = a.loss_total = fake
+        a.B, a.k, a.kt, a.V, a.v0, a.Vl, a.P, a.rank = 4, 8, 8, 1024, 0, 512, 2, 0
+        a.mode, a.temperature, a.distill, a.lambda_, a.clip_c, a.grad_scale = 0, 1.0, 1, 0.5, 1.0, 1.0
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return ctypes.byref(a)
+
+    bad = [dict(P=0), dict(rank=2), dict(rank=-1), dict(v0=600), dict(Vl=0), dict(k=33, kt=33),
+           dict(kt=10), dict(mode=1), dict(temperature=0.0), dict(lambda_=2.0),
+           dict(clip_c=-1.0), dict(distill=2), dict(D=None), dict(dlogits=None)]
+    for kw in bad:
+        assert L.svd_vs_stats(args(**kw), fake, ws, 1 << 20, None) == 1, kw
+        assert L.svd_vs_resolve(args(**kw), fake, fake, ws, 1 << 20, None) == 1, kw
+        assert L.svd_vs_finish(args(**kw), fake, ws, 1 << 20, None) == 1, kw
+    # buffers and workspace
+    assert L.svd_vs_stats(args(), None, ws, 1 << 20, None) == 1
+    assert L.svd_vs_resolve(args(), fake, None, ws, 1 << 20, None) == 1
+    assert L.svd_vs_finish(args(), None, ws, 1 << 20, None) == 1
+    assert L.svd_vs_stats(args(), fake, ctypes.c_void_p(0x10010), 1 << 20, None) == 2
+    assert L.svd_vs_stats(args(), fake, ws, 16, None) == 3
+    # empty batch: nothing to do
+    assert L.svd_vs_stats(args(B=0), None, None, 0, None) == 0
+    assert L.svd_vs_stats(None, fake, ws, 1 << 20, None) == 1
