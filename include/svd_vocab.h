@@ -31,8 +31,7 @@
  * Conventions as in svd.h: bf16 as uint16_t bits, device pointers, rows contiguous, every
  * call enqueues on `stream` and never synchronizes, argument errors are returned before any
  * launch, device errors (a draft token outside [0, V)) go to the workspace status word and are
- * read with svd_get_device_error(ws).  The workspace must be zero before its first use;
- * svd_vs_finish leaves its counters zero again.
+ * read with svd_get_device_error(ws).  The workspace must be zero before its first use.
  * Limits: 1 <= k <= 32, kt in {k, k+1}, 1 <= Vl, 0 <= v0, v0 + Vl <= V < 2^31, 1 <= P <= 64.
  * The slices of the P ranks must tile [0, V) (not checkable by one rank).  The fast path needs
  * Vl % 8 == 0 and 16-byte aligned D, T and dlogits; other slices take plain loads and stores.

@@ -26,7 +26,7 @@
 
 #include <cmath>
 
-#include "../../include/svd_vocab.h"
+#include "svd_vocab.h"
 #include "svd_device.cuh"
 #include "svd_internal.h"
 
@@ -508,7 +508,7 @@ template <bool ALIGNED>
 __global__ void __launch_bounds__(kVsThreads) vs_masses_kernel(const VsParams p) {
     __shared__ float redf[kVsWarps];
     __shared__ unsigned long long redu[kVsWarps];
-    const int row = blockIdx.x, t = threadIdx.x;
+    const int row = gridDim.x - 1 - blockIdx.x, t = threadIdx.x;   // reverse order, as finish
     const int b = row / p.kt, i = row % p.kt;
     const RowState s = p.rows[row];
     const bool clip = (s.flags & kRowClip) != 0, samp = (s.flags & kRowSample) != 0;
@@ -524,12 +524,13 @@ __global__ void __launch_bounds__(kVsThreads) vs_masses_kernel(const VsParams p)
     float cd = 0.f, cq = 0.f, nc = 0.f;
     unsigned long long m = 0ull, pm = 0ull;
     for (int g0 = t; g0 < nvec; g0 += kVsThreads * kVsUnroll) {
+        // a clip-only row needs T only where a vector of D passes the clip bound
         uint4 tv[kVsUnroll], dv[kVsUnroll];
 #pragma unroll
         for (int u = 0; u < kVsUnroll; ++u) {
             const int g = g0 + u * kVsThreads;
             if (g < nvec) {
-                tv[u] = load_vec<ALIGNED>(Trow, g, p.Vl);
+                if (samp) tv[u] = load_vec<ALIGNED>(Trow, g, p.Vl);
                 if (verified) dv[u] = load_vec<ALIGNED>(Drow, g, p.Vl);
             }
         }
@@ -538,13 +539,14 @@ __global__ void __launch_bounds__(kVsThreads) vs_masses_kernel(const VsParams p)
             const int g = g0 + u * kVsThreads;
             if (g >= nvec) break;
             float xt[8], xd[8];
-            unpack8(tv[u], xt);
+            if (samp) unpack8(tv[u], xt);
             if (verified) unpack8(dv[u], xd);
             if (clip) {
                 // d_v = q_v s_v <= q_v s_max: only a vector whose largest q passes c / s_max
                 // can hold clipped entries; those are tested exactly
                 const float qv = fast_exp2(__fsub_rn(__fmul_rn(max8_bf16(dv[u]), k2), s.L2D));
                 if (qv > s.qthr) {
+                    if (!samp) unpack8(load_vec<ALIGNED>(Trow, g, p.Vl), xt);
 #pragma unroll
                     for (int l = 0; l < 8; ++l) {
                         const float q = elem_q(xd[l], k2, s.L2D);
@@ -606,11 +608,13 @@ __device__ __forceinline__ void store_grad(const VsParams& p, size_t drow, int g
     }
 }
 
+// Rows run in the reverse of the stats pass's order, so the rows it read last (the ones most
+// likely still in L2) are read again first.
 template <bool ALIGNED, bool FP32>
-__global__ void __launch_bounds__(kVsThreads) vs_finish_kernel(const VsParams p) {
+__global__ void __launch_bounds__(kVsThreads, 3) vs_finish_kernel(const VsParams p) {
     __shared__ unsigned long long scan[kVsWarps];
     __shared__ int found;
-    const int row = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int row = gridDim.x - 1 - blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int b = row / p.kt, i = row % p.kt;
     const RowState s = p.rows[row];
     const bool verified = (s.flags & kRowVerified) != 0;

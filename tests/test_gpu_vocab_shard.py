@@ -108,6 +108,32 @@ def test_clipping_sharded(clip_c, lam):
                       step=0, lam=lam, clip_c=clip_c, grad_seqs=list(range(B)))
 
 
+@pytest.mark.parametrize("V,Pn,align", [(50001, 2, 1), (40000, 2, 8), (151936, 1, 8)])
+def test_long_slices_and_workspace_reuse(V, Pn, align):
+    # slices of 20000 to 151936 ids (ragged and aligned), then a second step on the same buffers
+    B, k = 3, 4
+    D, T = rand_case(B, k, k + 1, V, 21, sigma=0.6)
+    bk = torch.tensor([4, 2, 3], dtype=torch.int32)
+    out, _ = run_sharded(D, T, bk, Pn, align=align, lam=0.5, clip_c=0.2)
+    compare_sequences(out, D, T, None, bk.numpy(), list(range(B)), mode=0, tau=1.0, seed=0,
+                      step=0, lam=0.5, clip_c=0.2, grad_seqs=[0, 2])
+    draft = syn.sample_draft_tokens(D, 1.0, 2)
+    out, shards = run_sharded(D, T, bk, Pn, align=align, draft=draft, mode=api.STOCHASTIC,
+                              seed=9, step=0, lam=0.5, clip_c=0.2)
+    compare_sequences(out, D, T, draft, bk.numpy(), list(range(B)), mode=1, tau=1.0, seed=9,
+                      step=0, lam=0.5, clip_c=0.2, grad_seqs=[1])
+    # a second step on the same workspaces and exchange buffers
+    for s in shards:
+        s.set_step(1)
+    vp.run_emulated(shards)
+    torch.cuda.synchronize()
+    assert all(s.device_error() == 0 for s in shards)
+    out = dict(shards[0].outputs())
+    out["dlogits"] = torch.cat([s.dlogits for s in shards], dim=2)
+    compare_sequences(out, D, T, draft, bk.numpy(), list(range(B)), mode=1, tau=1.0, seed=9,
+                      step=1, lam=0.5, clip_c=0.2, grad_seqs=[1])
+
+
 def test_k32_bonus_row_and_verify_only():
     B, k, V = 5, 32, 640
     D, T = rand_case(B, k, k + 1, V, 3, sigma=0.05)   # near-identical rows: long accepted runs
