@@ -263,7 +263,7 @@ def time_vocab_shard(w, d, bk, bk_host, draft, P, stream, n=20):
     return {"P": P, "slice": Vl, "rank_step_ms": rank_ms, "stats_ms": part[0],
             "resolve_ms": part[1], "finish_ms": part[2],
             "rank_algorithmic_bytes": alg, "rank_hbm_gbs": alg / (rank_ms / 1000.0) / 1e9,
-            "exchange_bytes_per_rank": n1 + n2, "launches_per_rank_step": 5,
+            "exchange_bytes_per_rank": n1 + n2, "launches_per_rank_step": 4,
             "note": "all-gathers not timed (one GPU)"}
 
 

@@ -12,13 +12,14 @@
 //            their lowest ids, sum 2^(x k2 - round(m k2)) of D and T (online rescaling when a
 //            thread's maximum grows), sum e_v (D_v - T_v) (the reverse-KL moment), max(D - T),
 //            and D, T at the caller's token and D at the local target argmax.      -> Rec1
-//   resolve  one warp per sequence: every rank combines the P records of each row in rank
-//            order (identical arithmetic on every rank), takes the acceptance decisions and
+//   resolve  one CTA per sequence, one warp per row: every rank combines the P records of
+//            each row (identical arithmetic on every rank), takes the acceptance decisions and
 //            the b_k prefix, and keeps the row state in the workspace.  Then one CTA per row
 //            that needs it re-reads the slice for the clip sums (only vectors whose largest q
 //            can reach the clip bound) and the 2^-48 fixed-point sample masses.      -> Rec2
-//   finish   one CTA per row: the gradient slice from the combined sums, the loss rows, and
-//            on the rank whose mass interval holds the Philox target, the sample search.
+//   finish   one CTA per row: the gradient slice from the combined sums, the loss rows (the
+//            last CTA adds them up), and on the rank whose mass interval holds the Philox
+//            target, the sample search.
 //
 // Per-element arithmetic (q_v, p_v, s_v, d_v, the fixed-point masses) is the fused pass's
 // (svd_device.cuh), so every rank rounds an element the same way wherever it is recomputed.
@@ -77,7 +78,7 @@ struct alignas(16) SeqState {
 };
 
 struct VsLayout {
-    size_t rows, seqs, lrow, seq_loss, total;
+    size_t rows, seqs, lrow, total;
 };
 VsLayout vs_layout(int B, int k, int kt) {
     VsLayout L;
@@ -88,8 +89,6 @@ VsLayout vs_layout(int B, int k, int kt) {
     off = align256(off + sizeof(SeqState) * static_cast<size_t>(B));
     L.lrow = off;
     off = align256(off + sizeof(float) * static_cast<size_t>(B) * k);
-    L.seq_loss = off;
-    off = align256(off + sizeof(float) * static_cast<size_t>(B));
     L.total = off;
     return L;
 }
@@ -111,7 +110,6 @@ struct VsParams {
     RowState* rows;
     SeqState* seqs;
     float* lrow;
-    float* seq_loss;
     void* dlogits;
     float* loss_rows;
     float* loss_total;
@@ -328,9 +326,24 @@ __global__ void __launch_bounds__(kVsThreads) vs_stats_kernel(const VsParams p) 
 }
 
 // ------------------------------------------------------------------------------------------
-// resolve: one warp per sequence, lane i = row i (row 32, a bonus row only, on lane 0)
+// resolve: one CTA per sequence, one warp per row whose lanes read the ranks' records; warp 0
+// then takes the b_k prefix over the rows (row 32, a bonus row only, on warp 0's lane 0)
 // ------------------------------------------------------------------------------------------
+// (m, s, pos, aux) of another partial merged into this one: the larger maximum wins, equal
+// maxima keep the lower id, sums move onto the larger maximum's reference.
+__device__ __forceinline__ void merge_max(float& m, float& s, uint32_t& pos, float& aux, float m2,
+                                          float s2, uint32_t pos2, float aux2, float k2) {
+    const float M = fmaxf(m, m2);
+    s = s * rescale(m, M, k2) + s2 * rescale(m2, M, k2);
+    if (m2 > m || (m2 == m && pos2 < pos)) {
+        pos = pos2;
+        aux = aux2;
+    }
+    m = M;
+}
+
 __device__ RowState resolve_row(const VsParams& p, int b, int i, int n, bool& bad_token) {
+    const int lane = threadIdx.x & 31;
     RowState s;
     s.lseD = s.lseT = s.L2D = s.L2T = quiet_nan();
     s.dl = s.rkl = s.qthr = s.Dy = 0.f;
@@ -346,46 +359,52 @@ __device__ RowState resolve_row(const VsParams& p, int b, int i, int n, bool& ba
     const size_t stride = static_cast<size_t>(p.B) * p.kt;
     const size_t ri = static_cast<size_t>(b) * p.kt + i;
     const float k2 = p.k2, itau = p.itau;
-    float MD = neg_inf(), MT = neg_inf(), dmax = neg_inf();
-    for (int r = 0; r < p.P; ++r) {
-        const Rec1& a = p.recv1[r * stride + ri];
-        MD = fmaxf(MD, a.mD);
-        MT = fmaxf(MT, a.mT);
-        dmax = fmaxf(dmax, a.dmax);
-    }
-    uint32_t y = kNoId, xa = kNoId;
-    float sT = 0.f, sD = 0.f, sDd = 0.f, Dx = 0.f, Tx = 0.f;
-    for (int r = 0; r < p.P; ++r) {
-        const Rec1& a = p.recv1[r * stride + ri];
-        if (a.mT == MT) y = min(y, a.argT);
-        if (verified && a.mD == MD) xa = min(xa, a.argD);
-        sT += a.sT * rescale(a.mT, MT, k2);
+    // this lane's ranks (lane, lane + 32, ...), merged in rank order
+    float mD = neg_inf(), mT = neg_inf(), dmax = neg_inf();
+    float sD = 0.f, sDd = 0.f, sT = 0.f, Dx = 0.f, Tx = 0.f, Dy = 0.f, nil = 0.f;
+    uint32_t aD = kNoId, aT = kNoId;
+    for (int r = lane; r < p.P; r += 32) {
+        const Rec1 a = p.recv1[r * stride + ri];
+        merge_max(mT, sT, aT, Dy, a.mT, a.sT, a.argT, a.Dy, k2);
         if (verified) {
-            const float f = rescale(a.mD, MD, k2);
-            sD += a.sD * f;
-            sDd += a.sDd * f;
+            const float M = fmaxf(mD, a.mD);
+            sDd = sDd * rescale(mD, M, k2) + a.sDd * rescale(a.mD, M, k2);
+            merge_max(mD, sD, aD, nil, a.mD, a.sD, a.argD, 0.f, k2);
+            dmax = fmaxf(dmax, a.dmax);
             Dx += a.Dx;
             Tx += a.Tx;
         }
     }
-    float Dy = 0.f;
-    for (int r = 0; r < p.P; ++r) {
-        const Rec1& a = p.recv1[r * stride + ri];
-        if (a.argT == y) Dy = a.Dy;
-    }
+    // across the warp (a fixed butterfly order, the same on every rank)
+    const float MT = redux_max_f32(mT);
+    const uint32_t y = redux_min_u32(mT == MT ? aT : kNoId);
+    const uint32_t own = __ballot_sync(0xffffffffu, aT == y && y != kNoId);
+    s.Dy = __shfl_sync(0xffffffffu, Dy, own ? __ffs(own) - 1 : 0);
     s.y = y == kNoId ? -1 : static_cast<int32_t>(y);
-    s.Dy = Dy;
+    const float gsT = warp_sum(sT * rescale(mT, MT, k2));
+    float MD = neg_inf(), gsD = 0.f, gsDd = 0.f, gdmax = neg_inf(), gDx = 0.f, gTx = 0.f;
+    uint32_t xa = kNoId;
+    if (verified) {
+        MD = redux_max_f32(mD);
+        xa = redux_min_u32(mD == MD ? aD : kNoId);
+        const float f = rescale(mD, MD, k2);
+        gsD = warp_sum(sD * f);
+        gsDd = warp_sum(sDd * f);
+        gdmax = redux_max_f32(dmax);
+        gDx = warp_sum(Dx);      // one rank holds the caller's token, the others add exact zeros
+        gTx = warp_sum(Tx);
+    }
     const bool exps = (p.distill && verified) || p.stoch;
     float smax = 0.f;
     if (exps) {
-        s.lseT = MT * itau + logf(sT);
+        s.lseT = MT * itau + logf(gsT);
         s.L2T = s.lseT * kLog2e;
         if (verified) {
-            s.lseD = MD * itau + logf(sD);
+            s.lseD = MD * itau + logf(gsD);
             s.L2D = s.lseD * kLog2e;
             s.dl = s.lseD - s.lseT;
-            s.rkl = (sDd / sD) * itau - s.dl;          // sum_v q_v (log q_v - log p_v)
-            smax = dmax * itau - s.dl;                 // largest log q_v - log p_v
+            s.rkl = (gsDd / gsD) * itau - s.dl;        // sum_v q_v (log q_v - log p_v)
+            smax = gdmax * itau - s.dl;                // largest log q_v - log p_v
         }
     }
     if (verified) {
@@ -406,7 +425,7 @@ __device__ RowState resolve_row(const VsParams& p, int b, int i, int n, bool& ba
             const float u0 = uniform24(ph.w[0]);
             s.u1 = uniform24(ph.w[1]);
             if (x != kNoId) {
-                s.ratio = fast_exp2((s.dl - (Dx - Tx) * itau) * kLog2e);
+                s.ratio = fast_exp2((s.dl - (gDx - gTx) * itau) * kLog2e);
                 s.acc = u0 < fminf(1.f, s.ratio) ? 1 : 0;
             } else {
                 s.ratio = 0.f;
@@ -443,18 +462,33 @@ __device__ __forceinline__ svd_row_info row_info_of(const VsParams& p, const Row
     return r;
 }
 
-__global__ void __launch_bounds__(256) vs_resolve_kernel(const VsParams p) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int b = blockIdx.x * 8 + warp;
-    if (b >= p.B) return;
+__global__ void __launch_bounds__(1024) vs_resolve_kernel(const VsParams p) {
+    __shared__ RowState srow[33];
+    __shared__ int bad;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int b = blockIdx.x;
     const int k = p.k, kt = p.kt;
     const int n = vs_bk(p, b);
-    bool bad = false;
-    RowState s = resolve_row(p, b, lane, n, bad);      // lanes >= kt return an empty state
-    RowState s32;
+    if (threadIdx.x == 0) bad = 0;
+    __syncthreads();
+    for (int i = warp; i < kt; i += nw) {
+        bool badt = false;
+        const RowState s = resolve_row(p, b, i, n, badt);
+        if (lane == 0) {
+            srow[i] = s;
+            if (badt) bad = 1;
+        }
+    }
+    __syncthreads();
+    if (warp != 0) return;
+    if (lane == 0 && bad) set_device_error(&p.hdr->status, SVD_ERR_TOKEN_RANGE);
+    RowState s = srow[lane < kt ? lane : 0];
+    if (lane >= kt) {
+        s.flags = 0u;
+        s.acc = -1;
+    }
     const bool has32 = kt == 33;
-    if (has32) s32 = resolve_row(p, b, 32, n, bad);     // uniform call; only lane 0 keeps it
-    if (__any_sync(0xffffffffu, bad) && lane == 0) set_device_error(&p.hdr->status, SVD_ERR_TOKEN_RANGE);
+    RowState s32 = srow[has32 ? 32 : 0];
     // acceptance prefix: first verified row not accepted, else n
     const uint32_t accm = __ballot_sync(0xffffffffu, lane < n && s.acc == 1);
     int a = __ffs(~accm) - 1;
@@ -480,10 +514,9 @@ __global__ void __launch_bounds__(256) vs_resolve_kernel(const VsParams p) {
     }
     // emitted tokens: the accepted drafts, then the correction / bonus token (greedy: the
     // target argmax of that row; stochastic: written by the rank whose slice holds the draw)
-    const int xl = s.x;
-    if (lane < k + 1 && lane < 32) {
+    if (lane < k + 1) {
         int v = -1;
-        if (lane < a) v = xl;
+        if (lane < a) v = s.x;
         else if (lane == a && fix_row >= 0) v = fix_tok;
         p.emitted[static_cast<size_t>(b) * (k + 1) + lane] = v;
     }
@@ -613,7 +646,8 @@ __device__ __forceinline__ void store_grad(const VsParams& p, size_t drow, int g
 template <bool ALIGNED, bool FP32>
 __global__ void __launch_bounds__(kVsThreads, 3) vs_finish_kernel(const VsParams p) {
     __shared__ unsigned long long scan[kVsWarps];
-    __shared__ int found;
+    __shared__ float part[kVsThreads];
+    __shared__ int found, last;
     const int row = gridDim.x - 1 - blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int b = row / p.kt, i = row % p.kt;
     const RowState s = p.rows[row];
@@ -705,6 +739,35 @@ __global__ void __launch_bounds__(kVsThreads, 3) vs_finish_kernel(const VsParams
         }
     }
 
+    if (p.distill) {
+        // the last CTA to finish adds the loss rows: per sequence in row order, sequences in a
+        // fixed order (thread t takes sequences t, t + 256, ...; the threads in order)
+        __syncthreads();
+        if (t == 0) {
+            __threadfence();
+            last = atomicAdd(&p.hdr->loss_ticket, 1u) == gridDim.x - 1 ? 1 : 0;
+        }
+        __syncthreads();
+        if (last) {
+            __threadfence();
+            float acc = 0.f;
+            for (int bb = t; bb < p.B; bb += kVsThreads) {
+                const int nb = p.seqs[bb].n;
+                float ls = 0.f;
+                for (int q = 0; q < nb; ++q) ls += __ldcg(p.lrow + static_cast<size_t>(bb) * p.k + q);
+                acc += ls;
+            }
+            part[t] = acc;
+            __syncthreads();
+            if (t == 0) {
+                float tot = 0.f;
+                for (int j = 0; j < kVsThreads; ++j) tot += part[j];
+                *p.loss_total = tot;
+                p.hdr->loss_ticket = 0u;     // ready for the next call
+            }
+        }
+    }
+
     if (!(s.flags & kRowSample)) return;
     // the correction / bonus draw: the rank whose mass interval holds the target searches
     unsigned long long R = 0ull, before = 0ull, mine = 0ull;
@@ -775,21 +838,6 @@ __global__ void __launch_bounds__(kVsThreads, 3) vs_finish_kernel(const VsParams
         p.emitted[static_cast<size_t>(b) * (p.k + 1) + q.a] = found;
         if (p.row_info) p.row_info[row].sample_token = found;
     }
-}
-
-// loss total: sequence sums over rows in order, then the sequences in order
-__global__ void __launch_bounds__(256) vs_total_kernel(const VsParams p) {
-    for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
-        const int n = p.seqs[b].n;
-        float ls = 0.f;
-        for (int q = 0; q < n; ++q) ls += p.lrow[static_cast<size_t>(b) * p.k + q];
-        p.seq_loss[b] = ls;
-    }
-    __syncthreads();
-    if (threadIdx.x != 0) return;
-    float tot = 0.f;
-    for (int b = 0; b < p.B; ++b) tot += p.seq_loss[b];
-    *p.loss_total = tot;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -869,7 +917,6 @@ VsParams make_params(const svd_vs_args* a, void* ws) {
     p.rows = reinterpret_cast<RowState*>(base + L.rows);
     p.seqs = reinterpret_cast<SeqState*>(base + L.seqs);
     p.lrow = reinterpret_cast<float*>(base + L.lrow);
-    p.seq_loss = reinterpret_cast<float*>(base + L.seq_loss);
     p.dlogits = a->dlogits;
     p.loss_rows = a->loss_rows;
     p.loss_total = a->loss_total;
@@ -931,7 +978,7 @@ svd_status svd_vs_resolve(const svd_vs_args* a, const void* recv1, void* send2, 
     p.recv1 = static_cast<const Rec1*>(recv1);
     p.send2 = static_cast<Rec2*>(send2);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    vs_resolve_kernel<<<(a->B + 7) / 8, 256, 0, st>>>(p);
+    vs_resolve_kernel<<<a->B, 32 * (a->kt < 32 ? a->kt : 32), 0, st>>>(p);
     s = launched();
     if (s != SVD_OK) return s;
     const unsigned grid = static_cast<unsigned>(a->B) * a->kt;
@@ -957,9 +1004,6 @@ svd_status svd_vs_finish(const svd_vs_args* a, const void* recv2, void* ws, size
     else if (al) vs_finish_kernel<true, false><<<grid, kVsThreads, 0, st>>>(p);
     else if (f32) vs_finish_kernel<false, true><<<grid, kVsThreads, 0, st>>>(p);
     else vs_finish_kernel<false, false><<<grid, kVsThreads, 0, st>>>(p);
-    s = launched();
-    if (s != SVD_OK || !a->distill) return s;
-    vs_total_kernel<<<1, 256, 0, st>>>(p);
     return launched();
 }
 
