@@ -490,7 +490,8 @@ def main():
                          "avg_launch_ms": rows_avg_ms},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 3 * K,   # length head, row pass, finalize per step
+            # length head, row pass, finalize per step (+ the stochastic draw)
+            "gpu_launches": (4 if w.mode == 1 else 3) * K,
             "clocks": clock_rec,
             "accepted_tokens_per_s": red["accepted"] / (red["ms"] / 1000.0),
             "emitted_tokens_per_s": red["emitted"] / (red["ms"] / 1000.0),

@@ -73,7 +73,9 @@ typedef struct svd_row_info {
     int32_t draft_token;    /* x_i: caller token or argmax of the draft row; -1 if unverified */
     int32_t target_argmax;  /* argmax of the target row (verified rows and the bonus row)     */
     int32_t accepted;       /* 1 / 0 acceptance decision; -1 if the row was not verified      */
-    int32_t sample_token;   /* correction / bonus candidate drawn from this row; -1 if none   */
+    int32_t sample_token;   /* greedy: the target argmax of the row.  Stochastic: the drawn
+                             * correction / bonus token on the row it was drawn from (the
+                             * first rejected row, else the bonus row); -1 on other rows     */
     float ratio;            /* p_i(x_i) / q_i(x_i) in stochastic mode, NaN otherwise           */
     float lse_draft;        /* log sum_v exp(D_i,v / tau), NaN if not computed                */
     float lse_target;       /* log sum_v exp(T_i,v / tau), NaN if not computed                */

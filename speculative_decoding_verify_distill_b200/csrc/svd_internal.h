@@ -131,6 +131,8 @@ struct RowParams {
 // Launchers (return cudaError_t as int; 0 = success).
 int launch_length_head(const HeadParams& p, void* stream);
 int launch_row_pass(const RowParams& p, void* stream);
+// stochastic mode, after the finalize pass: each sequence's correction / bonus draw
+int launch_sample_fix(const RowParams& p, void* stream);
 int launch_wait_timeout_selftest(WsHeader* hdr, uint64_t limit_ns, void* stream);
 struct HeadUpdateParams {
     const uint16_t* h;

@@ -1,7 +1,7 @@
 // verify_distill.cu -- the fused row pass: truncated verification (greedy / stochastic) and the
-// clipped reverse-KL + CE distillation loss with its gradient, one HBM read per logit row; and the
+// clipped reverse-KL + CE distillation loss with its gradient, one HBM read per logit row; the
 // small finalize pass that turns per-row records into accepted lengths, emitted tokens and loss
-// sums.
+// sums; and, in stochastic mode, the draw of each sequence's correction or bonus token.
 //
 // What it computes (AdaFlash; Pith review page "What carries the argument", Axiom & Free-
 // Parameter Ledger, Referee Report major comment 2; Pith verdict record load_bearing_attack):
@@ -27,13 +27,17 @@
 //     sums, the reverse-KL moment sum e(D - T) and max(D - T).  Reduction #1 (warp -> CTA ->
 //     cluster over DSMEM) gives lse(D/tau), lse(T/tau) and the unclipped reverse-KL.
 //   * Pass B: only entries with q > c / max(log q - log p) can be clipped; those vectors alone
-//     are re-read and tested.  Stochastic rows take their sample masses here as 2^-48 fixed-point
-//     integers (exact, associative prefix sums).  Argmax (lowest id) is resolved lazily by the
-//     threads holding the row maximum.  Reduction #2.
+//     are re-read and tested.  Argmax (lowest id) is resolved lazily by the threads holding the
+//     row maximum.  Reduction #2 (only when some entry can be clipped).
 //   * Pass C: dL/dD = q (P + Q (D - T)) with the clipped and hard-label corrections, q
 //     recomputed from the staged logits, 16-byte streaming stores.
 //   * Rank 0 writes the row record after the next cluster barrier; the finalize kernel runs the
 //     warp-ballot acceptance scan per sequence and the fixed-order loss sums.
+//   * Stochastic mode: a sequence emits one drawn token, from its first rejected row (residual
+//     max(0, p - q)) or else its bonus row (p).  The row pass draws nothing; once the finalize
+//     pass knows the emitted row, one cluster per sequence takes that row's sample masses as
+//     2^-48 fixed-point integers (exact, associative prefix sums, so the split over CTAs does not
+//     change the draw) and the CTA holding the Philox target searches its slice in id order.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -60,21 +64,18 @@ struct alignas(16) Msg1 {          // after pass A
     float mD, sD, sDd, dmax;        // max D, sum 2^((D - mD) k2), sum of those times (D - T), max (D - T)
     float mT, sT;                   // max T, sum 2^((T - mT) k2)
     uint32_t argT, argD;            // lowest id holding mT / mD in the sender's slice
-    uint32_t prev_tok;              // token the sender sampled for the previous row, or none
     float prev_ce;                  // -log q_y of the previous row from the owner of y, else 0
     uint32_t next_item;             // rank 0: the cluster's next loaded item (packed)
-    uint32_t pad;
+    uint32_t pad0, pad1;
 };
-struct alignas(16) Msg2 {          // after pass B
-    float clip_d, clip_q, n_clip, pad0;    // clipped reverse-KL entries
-    unsigned long long mass;               // sample mass (2^-48 units)
-    unsigned long long pad1;
+struct alignas(16) Msg2 {          // after pass B: clipped reverse-KL entries
+    float clip_d, clip_q, n_clip, pad0;
 };
-static_assert(sizeof(Msg1) == 48 && sizeof(Msg2) == 32, "message sizes are multiples of 16 bytes");
+static_assert(sizeof(Msg1) == 48 && sizeof(Msg2) == 16, "message sizes are multiples of 16 bytes");
 // Row values rank 0 keeps until the record is written.
 struct Pending {
     int b, i, kind;
-    int x, y, acc, do_sample;
+    int x, y, acc;
     float ratio, lseD, lseT, kc;
 };
 
@@ -84,9 +85,7 @@ struct Ctl {
     Msg2 w2[NW];
     Msg1 in1[2][16];                // exchange #1 by row parity and sender rank
     Msg2 in2[16];                   // exchange #2 by sender rank
-    unsigned long long in3[16];     // fallback exchange (residual mass zero: sample from p)
-    uint64_t x1[2], x2, x3;         // exchange barriers
-    uint32_t my_tok[2];             // token sampled in this CTA, by row parity
+    uint64_t x1[2], x2;             // exchange barriers
     float my_ce[2];                 // -log q_y computed in this CTA, by row parity
     Pending pend;
     int wscan[NW];                  // prologue scan of the loaded-row counts
@@ -122,10 +121,9 @@ __device__ __forceinline__ Msg1 empty_msg1() {
     m.mD = m.mT = m.dmax = kNegInf;
     m.sD = m.sDd = m.sT = 0.f;
     m.argT = m.argD = kNone;
-    m.prev_tok = kNone;
     m.prev_ce = 0.f;
     m.next_item = 0u;
-    m.pad = 0u;
+    m.pad0 = m.pad1 = 0u;
     return m;
 }
 
@@ -247,9 +245,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         mbar_init(&c.x1[0], 1);
         mbar_init(&c.x1[1], 1);
         mbar_init(&c.x2, 1);
-        mbar_init(&c.x3, 1);
         fence_mbar_init();
-        c.my_tok[0] = c.my_tok[1] = kNone;
         c.my_ce[0] = c.my_ce[1] = 0.f;
         c.first_item = 0u;
     }
@@ -417,7 +413,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     uint32_t phase = 0;          // parity of this warp's staging barrier
     bool wait_dead = false;      // a bounded wait ran out: skip later waits so the kernel ends
     int it = 0;                  // loaded rows done (row parity selects the exchange #1 buffers)
-    uint32_t n2 = 0, n3 = 0;     // completed phases of exchange barriers #2 and #3
+    uint32_t n2 = 0;             // completed phases of exchange barrier #2
     bool pending = false;        // rank 0 owes the record of the previous loaded row
 
     auto wait_x = [&](uint64_t* bar, uint32_t parity) {
@@ -437,15 +433,14 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         }
     };
     // rank 0, one lane: the record of the previous loaded row
-    auto write_record = [&](uint32_t tok, float ce) {
+    // (stochastic rows: the one draw a sequence emits is made after the finalize pass)
+    auto write_record = [&](float ce) {
         const Pending& pd = c.pend;
         svd_row_info r;
         r.draft_token = pd.x;
         r.target_argmax = pd.y;
         r.accepted = pd.acc;
-        if (!verify) r.sample_token = -1;
-        else if (!STOCH) r.sample_token = pd.y;
-        else r.sample_token = (pd.do_sample && tok != kNone) ? static_cast<int32_t>(tok) : -1;
+        r.sample_token = (verify && !STOCH) ? pd.y : -1;
         r.ratio = pd.ratio;
         r.lse_draft = pd.lseD;
         r.lse_target = pd.lseT;
@@ -478,7 +473,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         const size_t trow = static_cast<size_t>(b) * kt + i;     // target row
         const bool isRow = (cur.kind == kItemRow);
         const bool rowVerify = isRow && verify;
-        // exps are needed for distillation rows and for stochastic sampling
+        // exps are needed for distillation rows and for the stochastic ratio and sampler (lse)
         const bool need_lse = (DISTILL && isRow) || STOCH;
 
         // caller's draft token and, in stochastic mode, D_x and T_x for the acceptance ratio
@@ -622,10 +617,9 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                     if (DISTILL) m.dmax = redux_max_f32(dmax);
                 }
             }
-            m.prev_tok = kNone;
             m.prev_ce = 0.f;
             m.next_item = 0u;
-            m.pad = 0u;
+            m.pad0 = m.pad1 = 0u;
             if (lane == 0) c.w1[warp] = m;
         }
         if (zunits > 0 && t == 0) c.zu[par] = zfetch;
@@ -651,17 +645,13 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 const int fw = static_cast<int>(__shfl_sync(0xffffffffu, fetched, 0));
                 nitem = pack_item(decode_loaded(p, list, bkv, fw, verify));
             }
-            // the previous row's deposits of this CTA go out with this row's message
-            const uint32_t ptok = c.my_tok[par ^ 1];
+            // the previous row's -log q_y (if this CTA owns its y) goes out with this row's message
             const float pce = c.my_ce[par ^ 1];
             send1(make_uint4(__float_as_uint(cmD), __float_as_uint(csD), __float_as_uint(csDd), __float_as_uint(cdmax)),
                   make_uint4(__float_as_uint(cmT), __float_as_uint(csT), cargT, cargD),
-                  make_uint4(ptok, __float_as_uint(pce), nitem, 0u), par);
+                  make_uint4(__float_as_uint(pce), nitem, 0u, 0u), par);
             __syncwarp();
-            if (lane == 0) {
-                c.my_tok[par ^ 1] = kNone;
-                c.my_ce[par ^ 1] = 0.f;
-            }
+            if (lane == 0) c.my_ce[par ^ 1] = 0.f;
         }
         if (zunits > 0) {
             const int zu = c.zu[par];
@@ -671,14 +661,13 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
 
         // ------------------------------------------------ row statistics (every warp)
         float MD, MT, lseD = kQNaN, lseT = kQNaN, L2D = 0.f, L2T = 0.f, dl = 0.f, rkl = 0.f, smax = 0.f;
-        uint32_t y, ptok_all;
+        uint32_t y;
         {
             const Msg1 a = lane < CL ? c.in1[par][lane] : empty_msg1();
             MD = redux_max_f32(a.mD);
             MT = redux_max_f32(a.mT);
             y = redux_min_u32(a.mT == MT ? a.argT : kNone);
             if (greedy_x && isRow) x = redux_min_u32(a.mD == MD ? a.argD : kNone);
-            ptok_all = redux_min_u32(a.prev_tok);
             if (compact) nxt = unpack_item(__shfl_sync(0xffffffffu, a.next_item, 0));
             if (need_lse) {
                 const float sT = warp_sum(a.sT * rescale(a.mT, MT, k2));
@@ -695,33 +684,28 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                     if (DISTILL) smax = redux_max_f32(a.dmax) * itau - dl;   // largest log q_v - log p_v
                 }
             }
-            // rank 0 writes the previous row's record (its token and -log q_y arrived just now)
+            // rank 0 writes the previous row's record (its -log q_y arrived just now)
             if (pending && rank == 0 && warp == NW - 1) {
                 const float pce = warp_sum(a.prev_ce);   // one owner sends it, the rest send 0
-                if (lane == 0) write_record(ptok_all, pce);
+                if (lane == 0) write_record(pce);
             }
         }
         pending = false;
 
-        // stochastic decision (every warp computes the same value)
-        float ratio = kQNaN, u1 = 0.f;
-        int acc = 0, do_sample = 0;
-        if (STOCH) {
+        // stochastic decision (every warp computes the same value); the correction or bonus
+        // token of a sequence is drawn after the finalize pass, from its one emitted row
+        float ratio = kQNaN;
+        int acc = 0;
+        if (STOCH && rowVerify) {
             const PhiloxOut ph = philox_words(p.seed, p.step, static_cast<uint32_t>(b),
                                               static_cast<uint32_t>(i));
             const float u0 = uniform24(ph.w[0]);
-            u1 = uniform24(ph.w[1]);
-            if (rowVerify) {
-                if (x != kNone) {
-                    ratio = fast_exp2((dl - (Dx - Tx) * itau) * kLog2e);
-                    acc = u0 < fminf(1.f, ratio) ? 1 : 0;
-                } else {
-                    ratio = 0.f;
-                    acc = 0;
-                }
-                do_sample = acc ? 0 : 1;
-            } else if (!isRow) {
-                do_sample = 1;  // bonus row: sample from p
+            if (x != kNone) {
+                ratio = fast_exp2((dl - (Dx - Tx) * itau) * kLog2e);
+                acc = u0 < fminf(1.f, ratio) ? 1 : 0;
+            } else {
+                ratio = 0.f;
+                acc = 0;
             }
         }
         if (rowVerify && !STOCH) acc = (x == y) ? 1 : 0;
@@ -735,7 +719,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             const float qmax = fast_exp2(__fsub_rn(__fmul_rn(MD, k2), L2D));
             do_clip = qmax * 1.001f > qthr;
         }
-        const bool need_x2 = do_clip || (STOCH && do_sample);
+        const bool need_x2 = do_clip;
 
         // -------------------------------------------------------- pass B
         // d_v = q_v s_v <= q_v s_max, so only entries with q_v > c / s_max can be clipped; those
@@ -761,90 +745,39 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 }
             }
         }
-        // stochastic rows: sample masses (residual max(0, p - q) of a rejected row, p of a bonus row)
-        unsigned long long vmass[NV];
-#pragma unroll
-        for (int j = 0; j < NV; ++j) vmass[j] = 0ull;
-        unsigned long long wmass = 0ull;
-        if (STOCH && do_sample) {
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                float xt[8];
-                unpack8(myT[j * 32 + lane], xt);
-                unsigned long long ms = 0ull;
-                if (isRow) {
-                    float xd[8];
-                    unpack8(myD[j * 32 + lane], xd);
-#pragma unroll
-                    for (int l = 0; l < 8; ++l)
-                        ms += to_fixed(fmaxf(__fsub_rn(elem_p(xt[l], k2, L2T), elem_q(xd[l], k2, L2D)), 0.f));
-                } else {
-#pragma unroll
-                    for (int l = 0; l < 8; ++l) ms += to_fixed(elem_p(xt[l], k2, L2T));
-                }
-                vmass[j] = ms;
-                wmass += ms;
-            }
-            wmass = warp_sum_u64(wmass);
-        }
-
-        // exchange #2: clip sums and sample masses (skipped when neither is needed)
+        // exchange #2: clip sums (skipped when no entry can be clipped)
         float g_clip_d = 0.f, g_clip_q = 0.f, g_n_clip = 0.f;
-        unsigned long long R = 0ull, before = 0ull;
-        // exclusive prefix of the sample masses of the warps before this one (this CTA)
-        auto warp_prefix = [&](unsigned long long m) -> unsigned long long {
-            unsigned long long incl = m;
-            warp_inclusive_scan_u64(incl);
-            return __shfl_sync(0xffffffffu, incl - m, warp);
-        };
         if (need_x2) {
             if (t == 0) mbar_arrive_expect_tx(&c.x2, static_cast<uint32_t>(CL * sizeof(Msg2)));
-            if (do_clip) {
-                clip_d = warp_sum(clip_d);
-                clip_q = warp_sum(clip_q);
-                n_clip = warp_sum(n_clip);
-            }
+            clip_d = warp_sum(clip_d);
+            clip_q = warp_sum(clip_q);
+            n_clip = warp_sum(n_clip);
             if (lane == 0) {
                 Msg2 q2;
                 q2.clip_d = clip_d; q2.clip_q = clip_q; q2.n_clip = n_clip; q2.pad0 = 0.f;
-                q2.mass = wmass;
-                q2.pad1 = 0ull;
                 c.w2[warp] = q2;
             }
             __syncthreads();
-            const unsigned long long mw = lane < NW ? c.w2[lane].mass : 0ull;
-            unsigned long long wpre = 0ull;
-            if (STOCH && do_sample) wpre = warp_prefix(mw);
             if (warp == 0) {
                 float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-                if (do_clip && lane < NW) {
+                if (lane < NW) {
                     a0 = c.w2[lane].clip_d; a1 = c.w2[lane].clip_q; a2 = c.w2[lane].n_clip;
                 }
-                if (do_clip) {
-                    a0 = warp_sum(a0);
-                    a1 = warp_sum(a1);
-                    a2 = warp_sum(a2);
-                }
-                const unsigned long long tot = warp_sum_u64(mw);
+                a0 = warp_sum(a0);
+                a1 = warp_sum(a1);
+                a2 = warp_sum(a2);
                 if (lane < CL) {
                     const uint32_t dst = dsmem_map(&c.in2[rank], static_cast<uint32_t>(lane));
                     const uint32_t bar = dsmem_map(&c.x2, static_cast<uint32_t>(lane));
                     st_async_v4(dst, make_uint4(__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2), 0u), bar);
-                    st_async_v4(dst + 16, make_uint4(static_cast<uint32_t>(tot), static_cast<uint32_t>(tot >> 32), 0u, 0u), bar);
                 }
             }
             wait_x(&c.x2, n2 & 1u);
             ++n2;
-            const Msg2 a = lane < CL ? c.in2[lane] : Msg2{0.f, 0.f, 0.f, 0.f, 0ull, 0ull};
-            if (do_clip) {
-                g_clip_d = warp_sum(a.clip_d);
-                g_clip_q = warp_sum(a.clip_q);
-                g_n_clip = warp_sum(a.n_clip);
-            }
-            if (STOCH && do_sample) {
-                R = warp_sum_u64(a.mass);
-                before = warp_sum_u64(lane < static_cast<int>(rank) ? a.mass : 0ull) + wpre;
-            }
+            const Msg2 a = lane < CL ? c.in2[lane] : Msg2{0.f, 0.f, 0.f, 0.f};
+            g_clip_d = warp_sum(a.clip_d);
+            g_clip_q = warp_sum(a.clip_q);
+            g_n_clip = warp_sum(a.n_clip);
         }
 
         // ------------------------------------------------ row results (every warp)
@@ -858,80 +791,6 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             Q = pre * (1.f - lam) * itau;
             Pc = pre * (lam - (1.f - lam) * S);
             hardc = pre * lam;
-        }
-
-        // stochastic fallback: residual mass zero -> sample from p (rare; one more exchange)
-        bool use_p = false;
-        if (STOCH && do_sample && R == 0ull && isRow) {
-            use_p = true;
-            if (t == 0) mbar_arrive_expect_tx(&c.x3, static_cast<uint32_t>(CL * sizeof(unsigned long long)));
-            wmass = 0ull;
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                float xt[8];
-                unpack8(myT[j * 32 + lane], xt);
-                unsigned long long ms = 0ull;
-#pragma unroll
-                for (int l = 0; l < 8; ++l) ms += to_fixed(elem_p(xt[l], k2, L2T));
-                vmass[j] = ms;
-                wmass += ms;
-            }
-            wmass = warp_sum_u64(wmass);
-            __syncthreads();   // every warp is done with the exchange #2 partials
-            if (lane == 0) c.w2[warp].mass = wmass;
-            __syncthreads();
-            const unsigned long long mw = lane < NW ? c.w2[lane].mass : 0ull;
-            const unsigned long long wpre = warp_prefix(mw);
-            if (warp == 0) {
-                const unsigned long long tot = warp_sum_u64(mw);
-                if (lane < CL)
-                    st_async_u64(dsmem_map(&c.in3[rank], static_cast<uint32_t>(lane)), tot,
-                                 dsmem_map(&c.x3, static_cast<uint32_t>(lane)));
-            }
-            wait_x(&c.x3, n3 & 1u);
-            ++n3;
-            const unsigned long long m = lane < CL ? c.in3[lane] : 0ull;
-            R = warp_sum_u64(m);
-            before = warp_sum_u64(lane < static_cast<int>(rank) ? m : 0ull) + wpre;
-        }
-
-        // -------------------------------------------------------- sample search
-        if (STOCH && do_sample && R > 0ull) {
-            const unsigned long long tgt = scale_mass(R, static_cast<uint32_t>(u1 * 16777216.0f));
-            unsigned long long run = before;   // mass before this lane's vector, id order
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                unsigned long long incl = vmass[j];
-                warp_inclusive_scan_u64(incl);
-                const unsigned long long lo = run + incl - vmass[j];
-                run += __shfl_sync(0xffffffffu, incl, 31);
-                if (j * 32 + lane < wcnt && vmass[j] > 0ull && lo <= tgt && tgt - lo < vmass[j]) {
-                    // the sample point lies in this vector: walk its 8 masses in id order
-                    const unsigned long long rel = tgt - lo;
-                    unsigned long long cum = 0ull;
-                    int pick = -1;
-                    float xt[8];
-                    unpack8(myT[j * 32 + lane], xt);
-                    if (isRow) {
-                        float xd[8];
-                        unpack8(myD[j * 32 + lane], xd);
-#pragma unroll
-                        for (int l = 0; l < 8; ++l) {
-                            const float pv = elem_p(xt[l], k2, L2T);
-                            cum += use_p ? to_fixed(pv) : to_fixed(fmaxf(__fsub_rn(pv, elem_q(xd[l], k2, L2D)), 0.f));
-                            if (pick < 0 && cum > rel) pick = l;
-                        }
-                    } else {
-#pragma unroll
-                        for (int l = 0; l < 8; ++l) {
-                            cum += to_fixed(elem_p(xt[l], k2, L2T));
-                            if (pick < 0 && cum > rel) pick = l;
-                        }
-                    }
-                    if (pick < 0) pick = 7;
-                    atomicMin(&c.my_tok[par], static_cast<uint32_t>(v0 + (wv0 + j * 32 + lane) * 8 + pick));
-                }
-            }
         }
 
         // -------------------------------------------------------- pass C: gradient row
@@ -1025,7 +884,6 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             pd.x = rowVerify ? (x == kNone ? -1 : static_cast<int>(x)) : -1;
             pd.y = static_cast<int>(y);
             pd.acc = rowVerify ? acc : -1;
-            pd.do_sample = do_sample;
             pd.ratio = ratio;
             pd.lseD = isRow ? lseD : kQNaN;
             pd.lseT = lseT;
@@ -1038,23 +896,21 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     }
     if (pending) {
         // uniform: every rank walked the same items.  One more exchange #1 carries the last
-        // row's sampled token and -log q_y to rank 0.
+        // row's -log q_y to rank 0.
         const int par = it & 1;
         if (t == 0) mbar_arrive_expect_tx(&c.x1[par], static_cast<uint32_t>(CL * sizeof(Msg1)));
         __syncthreads();
         if (warp == 0) {
-            const uint32_t ptok = c.my_tok[par ^ 1];
             const float pce = c.my_ce[par ^ 1];
             const uint32_t ninf = __float_as_uint(kNegInf);
             send1(make_uint4(ninf, 0u, 0u, ninf), make_uint4(ninf, 0u, kNone, kNone),
-                  make_uint4(ptok, __float_as_uint(pce), 0u, 0u), par);
+                  make_uint4(__float_as_uint(pce), 0u, 0u, 0u), par);
         }
         wait_x(&c.x1[par], static_cast<uint32_t>(it >> 1) & 1u);
         if (rank == 0 && warp == NW - 1) {
             const Msg1 a = lane < CL ? c.in1[par][lane] : empty_msg1();
-            const uint32_t ptok = redux_min_u32(a.prev_tok);
             const float pce = warp_sum(a.prev_ce);
-            if (lane == 0) write_record(ptok, pce);
+            if (lane == 0) write_record(pce);
         }
     }
 
@@ -1340,7 +1196,10 @@ int launch_row_pass(const RowParams& p, void* stream) {
     fc.dynamicSmemBytes = 0;
     fc.stream = static_cast<cudaStream_t>(stream);
     err = cudaLaunchKernelEx(&fc, finalize_kernel, q);
-    return static_cast<int>(err);
+    if (err != cudaSuccess) return static_cast<int>(err);
+    // stochastic verification: the one drawn token per sequence, once its row is known
+    if ((p.flags & kFlagStochastic) && (p.flags & kFlagVerify)) return launch_sample_fix(q, stream);
+    return 0;
 }
 
 }  // namespace svd
