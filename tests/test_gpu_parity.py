@@ -203,11 +203,28 @@ def test_stochastic_qwen_b64_sampled():
     st = compare_sequences(out, D, T, draft, bk, seqs, mode=1, tau=w.tau, seed=w.philox_seed,
                            step=0, lam=w.lam, clip_c=w.clip_c, grad_seqs=[5])
     print("stochastic near-ties:", st)
+    check_sample_rows(out, w)
     # the same workload with every b_k = k (full verification)
     out2 = run_fused(w, D, T, draft=draft, use_head=False, bk_in=torch.full((w.B,), w.k, dtype=torch.int32))
     compare_sequences(out2, D[:16], T[:16], draft, np.full(w.B, w.k, np.int32), seqs[:16], mode=1,
                       tau=w.tau, seed=w.philox_seed, step=0, lam=w.lam, clip_c=w.clip_c,
                       check_loss=False)
+
+
+def check_sample_rows(out, w):
+    """Stochastic rows: the drawn token sits on the row it was drawn from (the first rejected
+    row, else the bonus row) and equals the emitted one; every other row reports none."""
+    ri = ri_fields(out["row_info"])
+    acc = out["accept_len"].cpu().numpy()
+    bk = out["bk"].cpu().numpy()
+    em = out["emitted"].cpu().numpy()
+    for b in range(w.B):
+        a, nb = int(acc[b]), int(bk[b])
+        s = ri["sample_token"][b].copy()
+        if a < nb or nb < s.shape[0]:
+            assert s[a] == em[b, a] and 0 <= s[a] < w.V, (b, a, s[a], em[b, a])
+            s[a] = -1
+        assert (s == -1).all(), (b, a, ri["sample_token"][b])
 
 
 @pytest.mark.parametrize("clip_c,lam", syn.STRESS_SWEEP)
