@@ -544,8 +544,15 @@ __global__ void __launch_bounds__(kVsThreads) vs_masses_kernel(const VsParams p)
     const int row = gridDim.x - 1 - blockIdx.x, t = threadIdx.x;   // reverse order, as finish
     const int b = row / p.kt, i = row % p.kt;
     const RowState s = p.rows[row];
-    const bool clip = (s.flags & kRowClip) != 0, samp = (s.flags & kRowSample) != 0;
+    bool clip = (s.flags & kRowClip) != 0;
+    const bool samp = (s.flags & kRowSample) != 0;
     const bool verified = (s.flags & kRowVerified) != 0;
+    if (clip) {
+        // the vector test below, applied to this slice's maximum of D (from this rank's own
+        // record): if it fails, no vector of the slice can hold a clipped entry
+        const float mDown = p.recv1[static_cast<size_t>(p.rank) * p.B * p.kt + row].mD;
+        clip = fast_exp2(__fsub_rn(__fmul_rn(mDown, p.k2), s.L2D)) > s.qthr;
+    }
     if (!clip && !samp) {
         if (t == 0) p.send2[row] = Rec2{0.f, 0.f, 0.f, 0.f, 0ull, 0ull};
         return;
