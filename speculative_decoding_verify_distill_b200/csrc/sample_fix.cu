@@ -47,17 +47,20 @@ __device__ __forceinline__ uint4 row_vec(const uint16_t* row, int g, int V) {
     }
 }
 
-// The sample weight of each element of a vector pair, in 2^-48 units.
+// The sample weights of a vector's 8 elements in 2^-48 units: wp = p, and with `residual`
+// also wr = max(0, p - q).
 __device__ __forceinline__ void vec_masses(const uint4& tv, const uint4& dv, bool residual,
                                            float k2, float L2T, float L2D,
-                                           unsigned long long (&w)[8]) {
+                                           unsigned long long (&wp)[8],
+                                           unsigned long long (&wr)[8]) {
     float xt[8], xd[8];
     unpack8(tv, xt);
     if (residual) unpack8(dv, xd);
 #pragma unroll
     for (int l = 0; l < 8; ++l) {
         const float pv = elem_p(xt[l], k2, L2T);
-        w[l] = residual ? to_fixed(fmaxf(__fsub_rn(pv, elem_q(xd[l], k2, L2D)), 0.f)) : to_fixed(pv);
+        wp[l] = to_fixed(pv);
+        wr[l] = residual ? to_fixed(fmaxf(__fsub_rn(pv, elem_q(xd[l], k2, L2D)), 0.f)) : 0ull;
     }
 }
 
@@ -92,17 +95,10 @@ __global__ void __launch_bounds__(kFixThreads) sample_fix_kernel(const RowParams
     for (int g = gbeg + t; g < gend; g += kFixThreads) {
         const uint4 tv = row_vec<ALIGNED>(Trow, g, V);
         const uint4 dv = residual ? row_vec<ALIGNED>(Drow, g, V) : tv;
-        unsigned long long w[8];
-        vec_masses(tv, dv, residual, k2, L2T, L2D, w);
-        if (residual) {
-            unsigned long long wp[8];
-            vec_masses(tv, tv, false, k2, L2T, L2D, wp);
+        unsigned long long wp[8], wr[8];
+        vec_masses(tv, dv, residual, k2, L2T, L2D, wp, wr);
 #pragma unroll
-            for (int l = 0; l < 8; ++l) { m += w[l]; pm += wp[l]; }
-        } else {
-#pragma unroll
-            for (int l = 0; l < 8; ++l) pm += w[l];
-        }
+        for (int l = 0; l < 8; ++l) { m += wr[l]; pm += wp[l]; }
     }
     m = warp_sum_u64(m);
     pm = warp_sum_u64(pm);
@@ -139,14 +135,17 @@ __global__ void __launch_bounds__(kFixThreads) sample_fix_kernel(const RowParams
     unsigned long long run = 0ull;    // mass of this slice's vectors before the round, id order
     for (int r0 = gbeg; r0 < gend; r0 += kFixThreads) {
         const int g = r0 + t;
-        unsigned long long w[8];
+        unsigned long long w[8], wr[8];
         unsigned long long vm = 0ull;
         if (g < gend) {
             const uint4 tv = row_vec<ALIGNED>(Trow, g, V);
             const uint4 dv = res ? row_vec<ALIGNED>(Drow, g, V) : tv;
-            vec_masses(tv, dv, res, k2, L2T, L2D, w);
+            vec_masses(tv, dv, res, k2, L2T, L2D, w, wr);
 #pragma unroll
-            for (int l = 0; l < 8; ++l) vm += w[l];
+            for (int l = 0; l < 8; ++l) {
+                if (res) w[l] = wr[l];
+                vm += w[l];
+            }
         }
         unsigned long long incl = vm;
         warp_inclusive_scan_u64(incl);
