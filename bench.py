@@ -334,6 +334,9 @@ def main():
     fused()
     torch.cuda.synchronize()
     bk_host = bk.cpu().numpy()
+    # boundary cases: gamma * bhat * k within 1e-4 of an integer (ceil / floor decided by rounding)
+    bk_near = int((np.abs(fused.bhat.cpu().double().numpy() * w.k
+                          - np.round(fused.bhat.cpu().double().numpy() * w.k)) < 1e-4).sum())
     acc_host = fused.accept_len.cpu().numpy()
     ne_host = fused.n_emitted.cpu().numpy()
     # the step's speedup report (rho = 0: verification-count view of the pages' eta)
@@ -501,6 +504,7 @@ def main():
             "full_k_step_ms": fullk_ms,
             "full_k_step_hbm_gbs": fullk_bytes / (fullk_ms / 1000.0) / 1e9,
             "bk_hist": bk_hist,
+            "boundary_cases": {"bk_near_integer": bk_near},
             "vocab_sharded": vshard,
             "speedup_report": {k_: (None if v_ != v_ else round(v_, 6)) for k_, v_ in report.items()
                                if k_ != "alpha"},
