@@ -95,6 +95,18 @@ def test_small_stochastic_sharded(Pn, kt_extra):
                          lam=0.5, clip_c=1.0)
     compare_sequences(out, D, T, draft, bk.numpy(), list(range(B)), mode=1, tau=1.0, seed=77,
                       step=3, lam=0.5, clip_c=1.0, grad_seqs=[0, 5, 23])
+    # after the max-combine: the drawn token on its row (the first rejected row, else the
+    # bonus row), equal to the emitted one; no token on any other row
+    ri = ri_fields(out["row_info"])
+    acc = out["accept_len"].cpu().numpy()
+    em = out["emitted"].cpu().numpy()
+    for b in range(B):
+        a, nb = int(acc[b]), int(bk[b])
+        st = ri["sample_token"][b].copy()
+        if a < nb or nb < st.shape[0]:
+            assert st[a] == em[b, a] and 0 <= st[a] < V, (b, a, st[a], em[b, a])
+            st[a] = -1
+        assert (st == -1).all(), (b, ri["sample_token"][b])
 
 
 @pytest.mark.parametrize("clip_c,lam", [(0.02, 0.0), (0.1, 0.5), (float("inf"), 0.0), (0.0, 1.0)])
