@@ -91,6 +91,22 @@ def test_block_sizes(k, kt):
     assert (vd.n_emitted.cpu().numpy() == (k + 1 if kt == k + 1 else k)).all()
 
 
+@pytest.mark.parametrize("k,kt", [(1, 2), (32, 33), (5, 6)])
+def test_block_sizes_stochastic(k, kt):
+    # the draw lands on the first rejected row or, with every draft accepted, on the bonus row
+    # (row 32 when k = 32: the last emitted slot)
+    B, V = 6, 2048
+    D, T = make_case(B, k, kt, V, seed=k * 10 + kt, sigma=1.0)
+    for bk, DD in ((syn.random_bk(B, k, k + 3), D),
+                   (torch.full((B,), k, dtype=torch.int32), T[:, :k].contiguous())):
+        draft = syn.sample_draft_tokens_batched(DD, 1.0, k + kt)
+        vd = fused(DD, T, bk, draft=draft, mode=1, seed=5, step=2)
+        full_compare(vd, DD, T, bk, draft=draft, mode=1, seed=5, step=2)
+    assert (vd.accept_len.cpu().numpy() == k).all()        # draft == target: all accepted
+    assert (vd.n_emitted.cpu().numpy() == k + 1).all()     # ... and the bonus token drawn
+    assert (vd.emitted.cpu().numpy()[:, k] >= 0).all()
+
+
 @pytest.mark.parametrize("B", [4096, 4097])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_batch_size_boundary_of_the_compact_lists(B, mode):
