@@ -18,9 +18,10 @@ Which pins hold each function (see ``tests/test_oracle_*.py``):
                         a hand-derived one-unit case; three AdamW steps against torch.optim.AdamW.
   * ``speedup_report`` -- hand-counted small cases; all-accepted and all-rejected limits; the
                         closed form recovered from geometric accept lengths (i.i.d. rate A).
-  * ``philox``       -- parity unpinned against published known-answer vectors (none are
-                        available offline); held by uniformity / independence chi-square tests
-                        and by bit-exact agreement with the independent CUDA implementation.
+  * ``philox``       -- bit-exact agreement with cuRAND's Philox4x32-10: its host generator
+                        (CPU suite: both key words, counter words 0-2) and its device API
+                        (GPU suite: counter words 2-3 from 64-bit subsequences); uniformity,
+                        independence and avalanche tests.
 """
 from __future__ import annotations
 

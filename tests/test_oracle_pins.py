@@ -7,6 +7,7 @@ sign/index or a transposed operand fails at least one of them.
 import json
 import math
 import os
+import sys
 
 import numpy as np
 import pytest
@@ -432,3 +433,57 @@ def test_philox_key_avalanche(orc):
             a, b = orc.philox4x32_10(ctr, key), orc.philox4x32_10(ctr, k2)
             flips.append(sum(bin(int(x) ^ int(y)).count("1") for x, y in zip(a, b)))
         assert 60 < np.mean(flips) < 68, word
+
+
+def _curand_host_lib():
+    """libcurand (the CUDA toolkit's, or the one that ships with torch); None if absent."""
+    import ctypes
+    import glob
+    import os
+    cands = [os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "lib64", "libcurand.so")]
+    for sp in sys.path:
+        cands += sorted(glob.glob(os.path.join(sp, "nvidia", "curand", "lib", "libcurand.so*")))
+    for c in cands:
+        if os.path.exists(c):
+            try:
+                return ctypes.CDLL(c)
+            except OSError:
+                continue
+    return None
+
+
+def _curand_host_philox_blocks(lib, seed, first_block, nblocks):
+    """Raw 32-bit outputs of cuRAND's host-side Philox4x32-10 generator (public API, no GPU),
+    from output 4 * first_block on, as [nblocks, 4]."""
+    import ctypes
+    gen = ctypes.c_void_p()
+    CURAND_RNG_PSEUDO_PHILOX4_32_10 = 161
+    assert lib.curandCreateGeneratorHost(ctypes.byref(gen), CURAND_RNG_PSEUDO_PHILOX4_32_10) == 0
+    try:
+        assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+        assert lib.curandSetGeneratorOffset(gen, ctypes.c_ulonglong(4 * first_block)) == 0
+        out = (ctypes.c_uint * (4 * nblocks))()
+        assert lib.curandGenerate(gen, out, ctypes.c_size_t(4 * nblocks)) == 0
+    finally:
+        lib.curandDestroyGenerator(gen)
+    return np.array(out[:], dtype=np.uint32).reshape(nblocks, 4)
+
+
+def test_philox_matches_curand_host_generator(orc):
+    # An independent Philox4x32-10: cuRAND's host generator, keyed by the 64-bit seed.  Its
+    # output stream runs 65536 subsequences side by side: block j of four words is the bijection
+    # at counter (n_lo, n_hi, j mod 65536, 0) with n = j div 65536 (observed from its outputs).
+    # That pins both key words and counter words 0-2 of the oracle's implementation.
+    lib = _curand_host_lib()
+    if lib is None:
+        pytest.skip("libcurand not found")
+    for seed in (0, 1, 0x0123456789ABCDEF, 0xDEADBEEF12345678, 2 ** 64 - 1):
+        key = [seed & 0xFFFFFFFF, seed >> 32]
+        for j0, n in ((0, 64), (65530, 12), (5 * 65536 + 77, 4), ((1 << 40) + 12345, 3),
+                      ((1 << 48) + 7, 3), ((1 << 60) + (1 << 50) + 99, 2)):
+            got = _curand_host_philox_blocks(lib, seed, j0, n)
+            for q in range(n):
+                j = j0 + q
+                c = j >> 16
+                ref = orc.philox4x32_10([c & 0xFFFFFFFF, c >> 32, j & 0xFFFF, 0], key)
+                assert np.array_equal(got[q], ref), (hex(seed), j)
