@@ -135,19 +135,9 @@ __device__ __forceinline__ uint32_t dsmem_map(const void* local, uint32_t rank) 
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(local)), "r"(rank));
     return r;
 }
-__device__ __forceinline__ float dsmem_ld_f32(uint32_t a) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-    return v;
-}
 __device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-    return v;
-}
-__device__ __forceinline__ double dsmem_ld_f64(uint32_t a) {
-    double v;
-    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(a) : "memory");
     return v;
 }
 __device__ __forceinline__ void dsmem_st_f32(uint32_t a, float v) {
@@ -156,21 +146,13 @@ __device__ __forceinline__ void dsmem_st_f32(uint32_t a, float v) {
 __device__ __forceinline__ void dsmem_st_u32(uint32_t a, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
-__device__ __forceinline__ void dsmem_min_u32(uint32_t a, uint32_t v) {
-    asm volatile("red.shared::cluster.min.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-// Asynchronous 16-byte / 8-byte store into another CTA's shared memory (cluster addresses from
+// Asynchronous 16-byte store into another CTA's shared memory (cluster addresses from
 // dsmem_map), counted as transaction bytes on that CTA's mbarrier `bar`.
 __device__ __forceinline__ void st_async_v4(uint32_t a, const uint4& v, uint32_t bar) {
     asm volatile(
         "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1,%2,%3,%4}, [%5];"
         ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar)
         : "memory");
-}
-__device__ __forceinline__ void st_async_u64(uint32_t a, unsigned long long v, uint32_t bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];"
-                 ::"r"(a), "l"(v), "r"(bar)
-                 : "memory");
 }
 
 // Warp-wide max / min in one instruction (f32 form: sm_100a).
