@@ -82,15 +82,27 @@ __global__ void __launch_bounds__(kBack1Threads) head_back1_kernel(const HeadUpd
         }
         __syncthreads();
         if (live) {
-#pragma unroll 8
-            for (int r = warp; r < nb; r += kW) {   // this warp's sequences, in order
-                const float d = sdelta[r];
-                const size_t o = static_cast<size_t>(b0 + r) * p.M + m;
-                const float u = p.u[o];
-                const float ev = u > 0.f ? d * w2 : 0.f;
-                gw += d * fmaxf(u, 0.f);
-                gb += ev;
-                p.e[o] = ev;
+            // this warp's sequences in order, kGroup at a time: the group's loads are all issued
+            // before its stores (which the compiler may not move loads across)
+            constexpr int kGroup = 8;
+            for (int r0 = warp; r0 < nb; r0 += kW * kGroup) {
+                float u[kGroup];
+#pragma unroll
+                for (int q = 0; q < kGroup; ++q) {
+                    const int r = r0 + q * kW;
+                    u[q] = r < nb ? p.u[static_cast<size_t>(b0 + r) * p.M + m] : 0.f;
+                }
+#pragma unroll
+                for (int q = 0; q < kGroup; ++q) {
+                    const int r = r0 + q * kW;
+                    if (r < nb) {
+                        const float d = sdelta[r];
+                        const float ev = u[q] > 0.f ? d * w2 : 0.f;
+                        gw += d * fmaxf(u[q], 0.f);
+                        gb += ev;
+                        p.e[static_cast<size_t>(b0 + r) * p.M + m] = ev;
+                    }
+                }
             }
         }
         __syncthreads();
@@ -166,7 +178,22 @@ __global__ void __launch_bounds__(256) head_back2_kernel(const HeadUpdateParams 
         }
         __syncthreads();
     }
-    // AdamW epilogue on this thread's 4 x 4 block of W1
+    // AdamW epilogue on this thread's 4 x 4 block of W1: every master weight and moment is
+    // loaded before the first store, so the 48 loads are in flight together
+    float wm[4][4], mm[4][4], vv[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int m = m0 + 4 * ty + i;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int j = j0 + 4 * tx + jj;
+            const bool in = m < p.M && j < p.H;
+            const size_t o = static_cast<size_t>(m) * p.H + j;
+            wm[i][jj] = in ? p.W1m[o] : 0.f;
+            mm[i][jj] = in ? p.mW1[o] : 0.f;
+            vv[i][jj] = in ? p.vW1[o] : 0.f;
+        }
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int m = m0 + 4 * ty + i;
@@ -176,11 +203,10 @@ __global__ void __launch_bounds__(256) head_back2_kernel(const HeadUpdateParams 
             const int j = j0 + 4 * tx + jj;
             if (j >= p.H) continue;
             const size_t o = static_cast<size_t>(m) * p.H + j;
-            float mm = p.mW1[o], vv = p.vW1[o];
-            const float w = adamw(p.W1m[o], acc[i][jj], mm, vv, p);
+            const float w = adamw(wm[i][jj], acc[i][jj], mm[i][jj], vv[i][jj], p);
             p.W1m[o] = w;
-            p.mW1[o] = mm;
-            p.vW1[o] = vv;
+            p.mW1[o] = mm[i][jj];
+            p.vW1[o] = vv[i][jj];
             p.W1[o] = f32_to_bf16_rne(w);
         }
     }
