@@ -267,6 +267,30 @@ def time_vocab_shard(w, d, bk, bk_host, draft, P, stream, n=20):
             "note": "all-gathers not timed (one GPU)"}
 
 
+def profile_head(w, dev, warmup, steps):
+    """The length head and one online update of it at the workload's (B, H, M), no logits."""
+    h, W1, b1, w2, b2 = (t.to(dev) if torch.is_tensor(t) else t for t in syn.make_head(w))
+    ws = api.Workspace(w.B, w.k, w.k, w.M, device=dev)
+    trainer = api.LengthHeadTrainer(W1, b1, w2, b2, w.B)
+    label = torch.full((w.B,), 0.5, dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        api.svd_length_head(h, W1, b1, w2, b2, w.k, ws=ws)
+        trainer.step(h, label)
+    torch.cuda.synchronize()
+    out = {}
+    for name, fn in (("length_head_ms", lambda: api.svd_length_head(h, W1, b1, w2, b2, w.k, ws=ws)),
+                     ("length_head_update_ms", lambda: trainer.step(h, label))):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / steps
+    print(json.dumps({"profile": "length_head", "workload": w.name, "B": w.B, "H": w.H, "M": w.M, **out}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -278,6 +302,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-vocab-shard", action="store_true", help="skip the vocab-sharded leg")
+    ap.add_argument("--profile-head", action="store_true",
+                    help="profiling only: time the length head and its update at the workload's "
+                         "shape, without logits, and print their times")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(syn.WORKLOADS),
                     help="profiling only: the reported bench line is the default workload")
     args = ap.parse_args()
@@ -297,6 +324,9 @@ def main():
     torch.cuda.set_device(info.local_rank)
     dev = torch.device("cuda", info.local_rank)
     w = syn.WORKLOADS[args.workload]
+    if args.profile_head:
+        profile_head(w, dev, args.warmup, args.steps)
+        return
     wr, host, d = build_inputs(w, parallel.rank_seed(0, info.rank) if info.rank else 0, dev)
     stream = torch.cuda.current_stream(dev)
 
