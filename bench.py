@@ -15,6 +15,12 @@ over ranks.  Rank 0 prints one JSON line.
 
 `--impl reference` times the CPU oracle (fp64, all host cores) on a bounded sample of the same
 workload instead and prints the same line with "impl": "reference".
+
+Besides the metric, the line carries the row pass's roofline, the end-to-end rate with host
+buffers, the CPU oracle baseline, clocks sampled during the timed region, and the other legs of
+the path timed on the same inputs: the length head and its online update, the full-k label mode,
+the speedup report and one rank of the 8-way vocab-sharded pass.  `--workload` and
+`--profile-head` are for profiling runs only.
 """
 from __future__ import annotations
 
