@@ -293,8 +293,9 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_cluster_kernel(const 
         for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
         if (lane == 0 && b0 + r < p.B) p.zpart[static_cast<size_t>(mt) * p.B + b0 + r] = z;
     }
-    // the last of this block's unit tiles finishes its 16 sequences
-    __threadfence();
+    // the last of this block's unit tiles finishes its 16 sequences; the lanes that wrote
+    // partial logits fence them before the ticket, the lanes that read them after it
+    if (lane == 0) __threadfence();
     __syncthreads();
     if (t == 0) {
         const uint32_t old = atomicAdd(&p.tile_ticket[bt], 1u);
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_cluster_kernel(const 
     }
     __syncthreads();
     if (!flag) return;
-    __threadfence();
+    if (t < kHeadTileB) __threadfence();
     if (t < kHeadTileB && b0 + t < p.B) {
         const int b = b0 + t;
         float z = p.b2_dev ? *p.b2_dev : p.b2;
