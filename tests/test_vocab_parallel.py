@@ -93,8 +93,8 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_step_gloo():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_multi_rank_step_gloo(world):
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -108,13 +108,13 @@ def test_two_rank_step_gloo():
     emitted = []
     for rank, c0, c1, recv1, c2, recv2, em, ri in res:
         assert (c0, c1, c2) == ("stats", "resolve", "finish")
-        assert recv1 == [10] * 12 + [11] * 12          # rank r's records at block r
-        assert recv2 == [20] * 8 + [21] * 8
+        assert recv1 == sum(([10 + r] * 12 for r in range(world)), [])   # rank r at block r
+        assert recv2 == sum(([20 + r] * 8 for r in range(world)), [])
         emitted.append(em)
         for b in range(3):
             assert em[b][0] == 5 and em[b][1] == 100 + b   # max-combined sampled token
             assert ri[b][1] == 100 + b
-    assert emitted[0] == emitted[1]
+    assert all(e == emitted[0] for e in emitted)
 
 
 def test_single_process_step_is_local():
