@@ -1,4 +1,4 @@
-"""The vocab-sharded step's host plumbing on CPU: slice tiling, and two gloo ranks running
+"""The vocab-sharded step's host plumbing on CPU: slice tiling, and two or three gloo ranks running
 ``vocab_parallel.step`` over a fake of the three library calls.  The fake records what each
 call saw, so the test checks the order of calls and exchanges, that every rank's records land
 at its rank's block of the gathered buffers before the next call reads them, and the
