@@ -41,3 +41,17 @@ def test_too_few_warmup_steps_are_refused():
     r = _run("--impl", "reference", "--steps", "1", "--warmup", "2", timeout=120)
     assert r.returncode != 0
     assert "warmup" in r.stderr
+
+
+def test_algorithmic_bytes_by_hand():
+    # each byte once: a verified row reads D and T and writes its gradient (6V), an unverified
+    # row's gradient is zero-filled (2V), a bonus row reads T (2V); plus the per-sequence outputs
+    sys.path.insert(0, ROOT)
+    import bench
+    import numpy as np
+    V, k, kt = 10, 4, 5
+    # sequence 0: b_k = 1 -> 1 x 60 + 3 x 20 + bonus 20 = 140; sequence 1: b_k = 4 -> 240 + 20 = 260
+    outputs = 2 * 4 * (3 + k + 1 + k)
+    assert bench.algorithmic_bytes(np.array([1, 4]), k, kt, V) == 140 + 260 + outputs
+    # kt = k: no bonus row when b_k = k
+    assert bench.algorithmic_bytes(np.array([4]), k, k, V) == 240 + 4 * (3 + k + 1 + k)
