@@ -78,6 +78,8 @@ def _load():
     lib.orc_distill_f64.argtypes = lib.orc_distill.argtypes
     lib.orc_distill_f64.restype = i32
     lib.orc_row_stats_f64.argtypes = [P, i32, f64, P, P, P]
+    lib.orc_clip_band.argtypes = [P, P, P, i32, i32, i32, i32, f64, f64, f64, P, P, P, P]
+    lib.orc_clip_band.restype = i32
     lib.orc_sample_inverse_cdf.argtypes = [P, i32, f64, P]
     lib.orc_sample_inverse_cdf.restype = ctypes.c_int32
     lib.orc_expected_tokens.argtypes = [f64, i32]
@@ -224,6 +226,27 @@ def distill(D, T, bk, lam: float, clip_c: float, tau: float = 1.0, grad_scale: f
         raise ValueError("oracle distill: bad arguments")
     return dict(loss_rows=loss_rows, loss_total=float(tot[0]), dlogits=g, rkl_rows=rkl,
                 kc_rows=kc, ce_rows=ce)
+
+
+def clip_band(D, T, bk, clip_c: float, tau: float = 1.0, band_rel: float = 1e-5,
+              want_mask: bool = True):
+    """Entries whose clip decision d_v <= c is within fp32 error of flipping (see
+    ``orc_clip_band``).  D [B,k,V], T [B,kt,V] bf16; returns dict n_band [B,k] int32,
+    dS [B,k] and dK [B,k] (bounds of the effect of flipped decisions on S and on K_c), and
+    band [B,k,V] bool (or None)."""
+    Db, Tb = _bits(D), _bits(T)
+    B, k, V = Db.shape
+    kt = Tb.shape[1]
+    bka = np.ascontiguousarray(np.asarray(bk, dtype=np.int32))
+    n = np.zeros((B, k), np.int32)
+    dS = np.zeros((B, k), np.float64)
+    dK = np.zeros((B, k), np.float64)
+    m = np.zeros((B, k, V), np.uint8) if want_mask else None
+    rc = _load().orc_clip_band(_ptr(Db), _ptr(Tb), _ptr(bka), B, k, kt, V, float(clip_c),
+                               float(tau), float(band_rel), _ptr(n), _ptr(dS), _ptr(dK), _ptr(m))
+    if rc != 0:
+        raise ValueError("oracle clip_band: bad arguments")
+    return dict(n_band=n, dS=dS, dK=dK, band=None if m is None else m.astype(bool))
 
 
 def expected_tokens(A: float, k: int) -> float:

@@ -484,6 +484,70 @@ int orc_distill_f64(const double* D, const double* T, const int32_t* bk, int B, 
                          loss_rows, loss_total, dlogits, rkl_rows, kc_rows, ce_rows);
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* Near-clip entries (the parity band of R6).  The clip decision d_v <= c of an entry is an   */
+/* fp64 decision here and an fp32 one on the GPU; the two can differ only where d_v lies      */
+/* within the fp32 error of d_v = q_v s_v from c.  That error is at most a few units of 1e-6  */
+/* times q_v (1 + |s_v|) (relative error of q_v from exp and lse, absolute error of s_v from   */
+/* the two lse values), so an entry is "in the band" when                                      */
+/*     |d_v - c| < band_rel * q_v * (1 + |s_v|).                                               */
+/* Per verified row (i < b_k) this reports:                                                    */
+/*   n_band [B,k]  entries in the band;                                                        */
+/*   dS     [B,k]  sum over band entries of q_v |s_v + 1|: the most a flipped decision can     */
+/*                 move S = sum_v m_v q_v (s_v + 1);                                           */
+/*   dK     [B,k]  sum over band entries of |d_v - c|: the most flipped decisions can move     */
+/*                 K_c = sum_v min(d_v, c);                                                    */
+/*   band   [B,k,V] (nullable) 1 for band entries, else 0.                                     */
+/* Rows i >= b_k and c = +inf have no band.                                                    */
+/* ------------------------------------------------------------------------------------------ */
+int orc_clip_band(const uint16_t* D, const uint16_t* T, const int32_t* bk, int B, int k, int kt,
+                  int V, double clip_c, double tau, double band_rel, int32_t* n_band, double* dS,
+                  double* dK, uint8_t* band) {
+    if (k < 1 || (kt != k && kt != k + 1) || V < 1 || B < 0 || !(tau > 0.0)) return 1;
+    for (int b = 0; b < B; ++b) if (bk[b] < 1 || bk[b] > k) return 1;
+    const int finite_c = isfinite(clip_c);
+#pragma omp parallel
+    {
+        double* lq = (double*)malloc(sizeof(double) * (size_t)V);
+        double* lp = (double*)malloc(sizeof(double) * (size_t)V);
+        double* Dw = (double*)malloc(sizeof(double) * (size_t)V);
+        double* Tw = (double*)malloc(sizeof(double) * (size_t)V);
+#pragma omp for schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b) {
+            for (int i = 0; i < k; ++i) {
+                size_t row = (size_t)b * k + i;
+                size_t trow = (size_t)b * kt + i;
+                int32_t n = 0;
+                double s_bound = 0.0, k_bound = 0.0;
+                uint8_t* bm = band ? band + row * (size_t)V : NULL;
+                if (bm) memset(bm, 0, (size_t)V);
+                if (i < bk[b] && finite_c) {
+                    widen_row(D + row * (size_t)V, V, Dw);
+                    widen_row(T + trow * (size_t)V, V, Tw);
+                    row_log_softmax(Dw, V, tau, lq);
+                    row_log_softmax(Tw, V, tau, lp);
+                    for (int v = 0; v < V; ++v) {
+                        double q = exp(lq[v]);
+                        double s = lq[v] - lp[v];
+                        double d = q * s;
+                        if (fabs(d - clip_c) < band_rel * q * (1.0 + fabs(s))) {
+                            ++n;
+                            s_bound += q * fabs(s + 1.0);
+                            k_bound += fabs(d - clip_c);
+                            if (bm) bm[v] = 1;
+                        }
+                    }
+                }
+                n_band[row] = n;
+                dS[row] = s_bound;
+                dK[row] = k_bound;
+            }
+        }
+        free(lq); free(lp); free(Dw); free(Tw);
+    }
+    return 0;
+}
+
 /* Inverse-CDF sampler exposed for its brute-force pin (R14). */
 int32_t orc_sample_inverse_cdf(const double* w, int V, double u, double* margin_out) {
     return sample_inverse_cdf(w, V, u, margin_out);

@@ -6,6 +6,13 @@ Tolerances (stated once):
   * losses, lse and fp32 gradients: |gpu - oracle| <= max(ATOL, RTOL * |oracle|) with
     RTOL = 1e-3, ATOL = 1e-5 (fp32 accumulation against the fp64 oracle);
   * bf16 gradients: within one bf16 ulp of RNE(oracle), or within ATOL of the oracle;
+  * clip decisions: an entry whose d_v = q_v s_v lies within TIE_CLIP * q_v (1 + |s_v|) of c
+    (oracle values; the fp32 error of d_v is below a third of that) may be clipped on one side
+    and not on the other.  Such "band" entries are counted, left out of the element-wise
+    gradient comparison, and every other entry of the row is compared with the tolerance above
+    widened by the most their flips can move the row's sums: (scale/tau)(1 - lambda) q_u dS for
+    the gradient, (1 - lambda) dK for the row loss (dS, dK from oracle.clip_band).  Band
+    entries must stay under 1% of each row;
   * stochastic accept decisions: identical unless |u - p/q| < 1e-6 (oracle values);
   * sampled tokens: identical unless the oracle's sample point lies within 1e-6 * R of a
     running-sum boundary;
@@ -22,6 +29,8 @@ RTOL, ATOL = 1e-3, 1e-5
 TIE_U = 1e-6
 TIE_SAMPLE = 1e-6
 TIE_BK = 1e-4
+TIE_CLIP = 2e-5
+BAND_MAX_FRAC = 0.01
 
 
 def close_mask(gpu, ref, rtol=RTOL, atol=ATOL):
@@ -30,8 +39,12 @@ def close_mask(gpu, ref, rtol=RTOL, atol=ATOL):
     return np.abs(gpu - ref) <= np.maximum(atol, rtol * np.abs(ref))
 
 
-def assert_close(gpu, ref, what, rtol=RTOL, atol=ATOL, mask=None):
+def assert_close(gpu, ref, what, rtol=RTOL, atol=ATOL, mask=None, extra=None):
+    """|gpu - ref| <= max(atol, rtol |ref|) (+ extra, a per-element widening) where mask is set."""
     ok = close_mask(gpu, ref, rtol, atol)
+    if extra is not None:
+        d = np.abs(np.asarray(gpu, np.float64) - np.asarray(ref, np.float64))
+        ok = ok | (d <= np.maximum(atol, rtol * np.abs(np.asarray(ref, np.float64))) + extra)
     if mask is not None:
         ok = ok | ~mask
     if not ok.all():
@@ -55,11 +68,12 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return 2.0 ** (np.floor(np.log2(ax)) - 7)
 
 
-def assert_bf16_grad(gpu_bf16: torch.Tensor, ref: np.ndarray, what: str, mask=None):
+def assert_bf16_grad(gpu_bf16: torch.Tensor, ref: np.ndarray, what: str, mask=None, extra=None):
     g = gpu_bf16.detach().to(torch.float64).cpu().numpy()
     r = np.asarray(ref, np.float64)
     rr = bf16_round(r)
-    ok = (np.abs(g - rr) <= bf16_ulp(rr)) | (np.abs(g - r) <= ATOL)
+    e = 0.0 if extra is None else extra
+    ok = (np.abs(g - rr) <= bf16_ulp(rr) + e) | (np.abs(g - r) <= ATOL + e)
     if mask is not None:
         ok = ok | ~mask
     if not ok.all():
@@ -74,18 +88,18 @@ def bk_near_integer(bhat: np.ndarray, k: int, gamma: float = 1.0) -> np.ndarray:
     return np.abs(x - np.round(x)) < TIE_BK
 
 
-def near_clip_rows(D, T, bk, c: float, tau: float, seqs=None) -> np.ndarray:
-    """[B,k] mask of verified rows that hold an entry with |d_v - c| < 1e-5 * max(1, c): the
-    clip decision of such an entry is not fixed by fp32 arithmetic (counted, not compared)."""
-    B, k, V = D.shape
-    out = np.zeros((B, k), bool)
-    if not math.isfinite(c):
-        return out
-    for b in range(B):
-        n = int(bk[b])
-        for i in range(n):
-            lq = torch.log_softmax(D[b, i].double() / tau, -1)
-            lp = torch.log_softmax(T[b, i].double() / tau, -1)
-            d = lq.exp() * (lq - lp)
-            out[b, i] = bool(((d - c).abs() < 1e-5 * max(1.0, c)).any())
-    return out
+def clip_band(D, T, bk, c: float, tau: float, want_mask: bool = True) -> dict:
+    """Band entries of the verified rows (see the module docstring) from the oracle, with the
+    per-row fraction checked against BAND_MAX_FRAC."""
+    import oracle
+    cb = oracle.clip_band(D, T, bk, c, tau, TIE_CLIP, want_mask=want_mask)
+    V = D.shape[2]
+    worst = cb["n_band"].max() if cb["n_band"].size else 0
+    assert worst <= max(1.0, BAND_MAX_FRAC * V), ("clip band too wide for an element-wise comparison",
+                                        int(worst), V)
+    return cb
+
+
+def softmax_rows(X, tau: float) -> np.ndarray:
+    """q = softmax(X / tau) of bf16 rows in fp64 (the tolerance widening only)."""
+    return torch.softmax(X.double() / tau, -1).numpy()

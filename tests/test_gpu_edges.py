@@ -163,7 +163,10 @@ def test_clipping_extremes_fp32_grad(clip_c, lam):
     D, T = make_case(2, 3, 3, 2056, seed=21, sigma=2.0)
     bk = torch.tensor([3, 2], dtype=torch.int32)
     vd = fused(D, T, bk, lam=lam, clip_c=clip_c, dl_fp32=True, grad_scale=0.125)
-    full_compare(vd, D, T, bk, lam=lam, clip_c=clip_c, dl_fp32=True, grad_scale=0.125)
+    st = full_compare(vd, D, T, bk, lam=lam, clip_c=clip_c, dl_fp32=True, grad_scale=0.125)
+    # the element-wise comparison covers (almost) every entry of the verified rows, c = 0 included
+    print("clip c=%g: %d band entries, %d compared" % (clip_c, st["clip_band"], st["clip_compared"]))
+    assert st["clip_compared"] >= 0.99 * (st["clip_compared"] + st["clip_band"])
 
 
 def test_single_purpose_entry_points():

@@ -50,7 +50,7 @@ def compare_sequences(out, D, T, draft, bk_used, seqs, *, mode, tau, seed, step,
     em_g = out["emitted"].cpu().numpy()[seqs]
     ne_g = out["n_emitted"].cpu().numpy()[seqs]
     ri = ri_fields(out["row_info"])
-    stats = dict(u_ties=0, sample_ties=0)
+    stats = dict(u_ties=0, sample_ties=0, clip_band=0, clip_compared=0)
     k = D.shape[1]
     kt = T.shape[1]
     for j, b in enumerate(seqs):
@@ -87,9 +87,12 @@ def compare_sequences(out, D, T, draft, bk_used, seqs, *, mode, tau, seed, step,
         want_grad_for = set(grad_seqs or [])
         sub = [j for j, b in enumerate(seqs) if b in want_grad_for]
         r = oracle.distill(D, T, bk_s, lam, clip_c, tau, grad_scale, want_grad=False)
-        near = P.near_clip_rows(D, T, bk_s, clip_c, tau)
+        # clip decisions fp32 cannot fix: counted entries, bounded effect on the row sums
+        cb = P.clip_band(D, T, bk_s, clip_c, tau, want_mask=bool(sub))
+        stats["clip_band"] = int(cb["n_band"].sum())
+        stats["clip_compared"] = int(bk_s.sum()) * D.shape[2] - stats["clip_band"]
         lr_g = out["loss_rows"].cpu().numpy()[seqs]
-        P.assert_close(lr_g, r["loss_rows"], "loss_rows", mask=~near)
+        P.assert_close(lr_g, r["loss_rows"], "loss_rows", extra=(1.0 - lam) * cb["dK"])
         verified = np.arange(k)[None, :] < bk_s[:, None]
         lse_g = ri["lse_draft"][seqs][:, :k]
         P.assert_close(lse_g[verified], _oracle_lse(D, bk_s, tau)[verified], "lse_draft")
@@ -97,12 +100,17 @@ def compare_sequences(out, D, T, draft, bk_used, seqs, *, mode, tau, seed, step,
             b = seqs[j]
             rg = oracle.distill(D[j:j + 1], T[j:j + 1], bk_s[j:j + 1], lam, clip_c, tau, grad_scale)
             g = out["dlogits"][b].cpu()
-            rowmask = np.ones_like(rg["dlogits"][0], bool)
-            rowmask[near[j]] = False
+            keep = ~cb["band"][j]
+            extra = None
+            if cb["n_band"][j].any():
+                q = P.softmax_rows(D[j], tau)
+                extra = (grad_scale / tau) * (1.0 - lam) * q * cb["dS"][j][:, None]
             if dl_fp32:
-                P.assert_close(g.numpy(), rg["dlogits"][0], "dlogits fp32 seq %d" % b, mask=rowmask)
+                P.assert_close(g.numpy(), rg["dlogits"][0], "dlogits fp32 seq %d" % b, mask=keep,
+                               extra=extra)
             else:
-                P.assert_bf16_grad(g, rg["dlogits"][0], "dlogits bf16 seq %d" % b, mask=rowmask)
+                P.assert_bf16_grad(g, rg["dlogits"][0], "dlogits bf16 seq %d" % b, mask=keep,
+                                   extra=extra)
     return stats
 
 
@@ -135,14 +143,19 @@ def run_fused(w: syn.Workload, D, T, *, draft=None, use_head=True, bk_in=None, l
 
 
 def check_bk(out, w: syn.Workload):
+    """b_k bit-exact against the oracle except at counted near-integers of gamma*bhat*k, which
+    must stay rare (at most 1% of the batch, and at least one allowed)."""
     h, W1, b1, w2, b2 = syn.make_head(w)
     bhat_ref, bk_ref, _ = oracle.length_head(h, W1, b1, w2, b2, w.k, 1.0, 0)
     bk_gpu = out["bk"].cpu().numpy()
     bhat_gpu = out["bhat"].cpu().numpy()
     near = P.bk_near_integer(bhat_ref, w.k)
+    n_near = int(near.sum())
+    print("%s: b_k near an integer (excluded from the exact check): %d of %d" % (w.name, n_near, w.B))
+    assert n_near <= max(1, w.B // 100), n_near
     assert np.array_equal(bk_gpu[~near], bk_ref[~near])
     P.assert_close(bhat_gpu, bhat_ref, "bhat", rtol=1e-4, atol=1e-6)
-    return bk_gpu, int(near.sum())
+    return bk_gpu, n_near
 
 
 # ------------------------------------------------------------------------------------------

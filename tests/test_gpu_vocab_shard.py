@@ -109,15 +109,19 @@ def test_small_stochastic_sharded(Pn, kt_extra):
         assert (st == -1).all(), (b, ri["sample_token"][b])
 
 
-@pytest.mark.parametrize("clip_c,lam", [(0.02, 0.0), (0.1, 0.5), (float("inf"), 0.0), (0.0, 1.0)])
+@pytest.mark.parametrize("clip_c,lam", [(0.02, 0.0), (0.1, 0.5), (float("inf"), 0.0), (0.0, 1.0),
+                                        (0.0, 0.0), (1e-4, 0.3)])
 def test_clipping_sharded(clip_c, lam):
     # wide noise makes many entries reach the clip bound
     B, k, V = 6, 4, 3000
     D, T = rand_case(B, k, k, V, 5, sigma=3.0)
     bk = torch.tensor([1, 2, 3, 4, 4, 2], dtype=torch.int32)
     out, _ = run_sharded(D, T, bk, 3, lam=lam, clip_c=clip_c, temperature=0.8)
-    compare_sequences(out, D, T, None, bk.numpy(), list(range(B)), mode=0, tau=0.8, seed=0,
-                      step=0, lam=lam, clip_c=clip_c, grad_seqs=list(range(B)))
+    st = compare_sequences(out, D, T, None, bk.numpy(), list(range(B)), mode=0, tau=0.8, seed=0,
+                           step=0, lam=lam, clip_c=clip_c, grad_seqs=list(range(B)))
+    print("sharded clip c=%g: %d band entries, %d compared" % (clip_c, st["clip_band"],
+                                                               st["clip_compared"]))
+    assert st["clip_compared"] >= 0.99 * (st["clip_compared"] + st["clip_band"])
 
 
 @pytest.mark.parametrize("V,Pn,align", [(50001, 2, 1), (40000, 2, 8), (151936, 1, 8)])

@@ -177,6 +177,47 @@ def test_clipping_invariants(orc):
     assert np.allclose(prev, rk, rtol=1e-14)                  # c beyond every entry: plain RKL
 
 
+def test_clip_band_special_cases(orc):
+    """The parity band of the clip decision (entries with |d_v - c| < eps q_v (1 + |s_v|)),
+    pinned on cases whose d_v are known in closed form."""
+    # D = [0, 0], T = [1, 0]: q = (1/2, 1/2), s1 = log((1 + e)/2), d1 = s1 / 2 (hand-derived)
+    e = math.e
+    s1 = math.log((1 + e) / 2)
+    d1 = s1 / 2
+    D = bf16(np.array([0.0, 0.0]).reshape(1, 1, 2))
+    T = bf16(np.array([1.0, 0.0]).reshape(1, 1, 2))
+    cb = orc.clip_band(D, T, [1], d1, 1.0, 2e-5)
+    assert cb["n_band"].tolist() == [[1]] and cb["band"][0, 0].tolist() == [False, True]
+    assert cb["dS"][0, 0] == pytest.approx(0.5 * abs(s1 + 1), rel=1e-12)
+    assert cb["dK"][0, 0] < 1e-15
+    for c in (d1 * (1 + 1e-3), d1 * (1 - 1e-3), 0.0, math.inf):
+        assert orc.clip_band(D, T, [1], c, 1.0, 2e-5)["n_band"][0, 0] == 0, c
+    assert orc.clip_band(D, T, [1], d1, 1.0, 0.0)["n_band"][0, 0] == 0   # empty band
+    # D = T: every s_v = 0, so at c = 0 every entry lies on the boundary; S moves by sum q = 1
+    Dq, _ = _rand_rows(11, 2, 3, 97)
+    cb = orc.clip_band(Dq, Dq, [3, 1], 0.0, 0.8, 2e-5)
+    assert cb["n_band"].tolist() == [[97, 97, 97], [97, 0, 0]]      # rows past b_k have none
+    assert np.allclose(cb["dS"][0], 1.0, rtol=1e-12) and cb["dS"][1, 1:].max() == 0.0
+    assert cb["dK"].max() == 0.0
+    assert orc.clip_band(Dq, Dq, [3, 1], 1e-3, 0.8, 2e-5)["n_band"].max() == 0
+
+
+def test_clip_band_brackets_decision_flips(orc):
+    """An entry whose d_v equals c (fp64, computed here by torch) is in the band of its row."""
+    D, T = _rand_rows(12, 2, 4, 512, sigma=2.0)
+    bk = [4, 3]
+    lq = F.log_softmax(D.double(), -1).numpy()
+    lp = F.log_softmax(T.double(), -1).numpy()
+    d = np.exp(lq) * (lq - lp)
+    for b, n in enumerate(bk):
+        for i in range(n):
+            c = float(np.sort(d[b, i])[-3])          # an entry sits exactly on the clip bound
+            cb = orc.clip_band(D[b:b + 1, i:i + 1], T[b:b + 1, i:i + 1], [1], c, 1.0, 2e-5)
+            v = int(np.argmax(d[b, i] == c))
+            assert cb["band"][0, 0, v]
+            assert cb["n_band"][0, 0] >= 1
+
+
 def test_rows_beyond_bk_are_zero(orc):
     D, T = _rand_rows(5, 3, 6, 50)
     bk = [1, 3, 6]
