@@ -162,25 +162,51 @@ def build_inputs(w: syn.Workload, seed_offset: int, dev):
     return wr, host, devd
 
 
-def cpu_oracle_sample(w: syn.Workload, host, n_seqs: int, threads: int, target_s: float = 10.0):
+def cpu_oracle_sample(w: syn.Workload, host, n_seqs: int, threads: int, target_s: float = 10.0,
+                      draft=None, bk_gpu=None):
     """Times the oracle (a1..a5, fp64) on the first n_seqs sequences, repeated until about
-    target_s seconds of CPU work have been timed; returns (tokens/s, info)."""
+    target_s seconds of CPU work have been timed; returns (tokens/s, info).
+
+    The same oracle calls also count, on that sample, the boundary cases the parity readings
+    exclude from exact comparison: stochastic accept tests with |u - p/q| < 1e-6, draws whose
+    sample point lies within 1e-6 R of a running-sum boundary, and clip decisions within the
+    fp32 band of the clip bound (entries with |d_v - c| < 2e-5 q_v (1 + |s_v|)).  With bk_gpu
+    (the GPU's b_k) the counts use the lengths the GPU verified."""
     import oracle
     oracle.build()
     oracle.set_threads(threads)
     seqs = list(range(n_seqs))
     D, T = host["D"][seqs], host["T"][seqs]
     h = host["h"][seqs]
+    dr = None if draft is None else draft[seqs].numpy()
     total, verified, reps = 0.0, 0, 0
+    ref = None
     while total < target_s and reps < 64:
         t0 = time.perf_counter()
         _, bk, _ = oracle.length_head(h, host["W1"], host["b1"].double().numpy(), host["w2"], host["b2"], w.k)
-        oracle.verify(D, T, None, bk, w.mode, w.tau, w.philox_seed, 0, seq_ids=seqs)
+        ref = oracle.verify(D, T, dr, bk, w.mode, w.tau, w.philox_seed, 0, seq_ids=seqs)
         oracle.distill(D, T, bk, w.lam, w.clip_c, w.tau, 1.0, want_grad=True)
         total += time.perf_counter() - t0
         verified += int(bk.sum())
         reps += 1
-    return verified / total, dict(seconds=total, verified=verified, seqs=n_seqs, reps=reps)
+    bk_c = np.asarray(bk if bk_gpu is None else bk_gpu[seqs], np.int32)
+    if bk_gpu is not None:
+        ref = oracle.verify(D, T, dr, bk_c, w.mode, w.tau, w.philox_seed, 0, seq_ids=seqs)
+    cases = {"sample": "first %d sequences, %d verified rows" % (n_seqs, int(bk_c.sum()))}
+    if w.mode == 1:
+        ver = np.arange(w.k)[None, :] < bk_c[:, None]
+        margin = np.abs(ref["row_u"] - np.minimum(1.0, ref["row_ratio"]))
+        cases["u_near_ratio"] = int((ver & (margin < 1e-6)).sum())
+        draws = ref["n_emitted"] > ref["accept_len"]
+        cases["sample_near_boundary"] = int((draws & (ref["fix_margin"] < 1e-6)).sum())
+    else:
+        cases["u_near_ratio"] = 0          # greedy: no uniform is drawn
+        cases["sample_near_boundary"] = 0
+    cb = oracle.clip_band(D, T, bk_c, w.clip_c, w.tau, 2e-5, want_mask=False)
+    cases["clip_band_entries"] = int(cb["n_band"].sum())
+    cases["clip_entries"] = int(bk_c.sum()) * w.V
+    return verified / total, dict(seconds=total, verified=verified, seqs=n_seqs, reps=reps,
+                                  cases=cases)
 
 
 def run_reference(args, info):
@@ -308,6 +334,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-vocab-shard", action="store_true", help="skip the vocab-sharded leg")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the headline workload (no legs for the other configs)")
     ap.add_argument("--profile-head", action="store_true",
                     help="profiling only: time the length head and its update at the workload's "
                          "shape, without logits, and print their times")
@@ -333,15 +361,45 @@ def main():
     if args.profile_head:
         profile_head(w, dev, args.warmup, args.steps)
         return
+    headline = run_leg(w, args, info, dev, headline=True)
+    legs = {}
+    # the other configurations on one GPU only (under torchrun every rank would regenerate them)
+    if not args.headline_only and info.world == 1:
+        for name in ("greedy_qwen_b32", "stochastic_qwen_b64", "stress_llama_b256"):
+            if name == args.workload:
+                continue
+            sweep = syn.STRESS_SWEEP if name == "stress_llama_b256" else None
+            legs[name] = run_leg(syn.WORKLOADS[name], args, info, dev, headline=False, sweep=sweep)
+    if info.rank == 0:
+        line = headline
+        line["legs"] = legs or None
+        # the boundary cases of every workload timed, counted on its oracle sample
+        cases = {args.workload: line.pop("_cases")}
+        for name, leg in legs.items():
+            cases[name] = leg.pop("_cases")
+        line["boundary_cases"] = cases
+        print(json.dumps(line), flush=True)
+    if info.world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def run_leg(w, args, info, dev, *, headline: bool, sweep=None):
+    """One workload: the fused step timed over K steps (with clocks on the headline), the row
+    pass alone (roofline), the end-to-end rate with host buffers and the CPU oracle sample.
+    The headline leg adds the head update, full-k mode, the speedup report and the sharded pass;
+    a sweep times the step again for each (c, lambda)."""
     wr, host, d = build_inputs(w, parallel.rank_seed(0, info.rank) if info.rank else 0, dev)
     stream = torch.cuda.current_stream(dev)
 
     ws = api.Workspace(w.B, w.k, w.kt, w.M, device=dev)
+    draft_host = None
     draft = None
     if w.mode == 1:
-        draft = syn.sample_draft_tokens(host["D"], w.tau, 77).to(dev)
+        draft_host = syn.sample_draft_tokens(host["D"], w.tau, 77)
+        draft = draft_host.to(dev)
     head = (d["h"], d["W1"], d["b1"], d["w2"], d["b2"])
-    # the product call: length head + row pass in one svd_verify_distill (programmatic launch)
+    # the product call: length head + row pass in one svd_verify_distill
     fused = api.VerifyDistill(d["D"], d["T"], head=head, draft_tok=draft, mode=w.mode,
                               temperature=w.tau, seed=w.philox_seed, lam=w.lam, clip_c=w.clip_c,
                               ws=ws)
@@ -366,13 +424,13 @@ def main():
         rows_only()
     torch.cuda.synchronize()
     if api.svd_get_device_error(ws) != 0:
-        raise SystemExit("device error during warm-up")
+        raise SystemExit("device error during warm-up (%s)" % w.name)
     fused()
     torch.cuda.synchronize()
     bk_host = bk.cpu().numpy()
     # boundary cases: gamma * bhat * k within 1e-4 of an integer (ceil / floor decided by rounding)
-    bk_near = int((np.abs(fused.bhat.cpu().double().numpy() * w.k
-                          - np.round(fused.bhat.cpu().double().numpy() * w.k)) < 1e-4).sum())
+    bhat_h = fused.bhat.cpu().double().numpy()
+    bk_near = int((np.abs(bhat_h * w.k - np.round(bhat_h * w.k)) < 1e-4).sum())
     acc_host = fused.accept_len.cpu().numpy()
     ne_host = fused.n_emitted.cpu().numpy()
     # the step's speedup report (rho = 0: verification-count view of the pages' eta)
@@ -380,7 +438,7 @@ def main():
 
     # ---------------------------------------------------------------- timed region (device)
     K = args.steps
-    clocks = None if args.no_clocks else ClockSampler(dev.index if dev.index is not None else 0)
+    clocks = None if (args.no_clocks or not headline) else ClockSampler(dev.index if dev.index is not None else 0)
     if info.world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -394,7 +452,7 @@ def main():
     t_end.record(stream)
     torch.cuda.synchronize()
     # per-kernel durations: the same step as two separately timed launches
-    KB = 200   # separate launches for the per-kernel times (outside the timed region)
+    KB = 200 if headline else 50   # separate launches for the per-kernel times (outside the timed region)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(KB)]
     for s in range(KB):
         ev[s][0].record(stream)
@@ -412,7 +470,7 @@ def main():
     ms_per_step = total_ms / K
     err = api.svd_get_device_error(ws)
     if err != 0:
-        raise SystemExit("device error in the timed region: %s" % api.STATUS_NAMES.get(err))
+        raise SystemExit("device error in the timed region (%s): %s" % (w.name, api.STATUS_NAMES.get(err)))
     vd = fused
 
     verified = float(bk_host.sum())
@@ -422,53 +480,86 @@ def main():
     red = parallel.reduce_metrics(ms_per_step, verified, accepted, emitted, loss, device=dev)
     value = red["verified"] / (red["ms"] / 1000.0)
 
-    # ---------------------------------------------------------------- length-head online update
-    trainer = api.LengthHeadTrainer(d["W1"], d["b1"], d["w2"], d["b2"], w.B)
-    label = (fused.accept_len.float() / bk.float()).contiguous()   # the proxy label a / b_k
-    for _ in range(3):
-        trainer.step(d["h"], label)
-    torch.cuda.synchronize()
-    u0 = torch.cuda.Event(enable_timing=True)
-    u1 = torch.cuda.Event(enable_timing=True)
-    n_upd = 50
-    u0.record(stream)
-    for _ in range(n_upd):
-        trainer.step(d["h"], label)
-    u1.record(stream)
-    torch.cuda.synchronize()
-    update_ms = u0.elapsed_time(u1) / n_upd
-
-    # ---------------------------------------------------------------- full-k label mode
-    # the same step verifying and distilling all k rows (labels a/b_k and a/k both observable)
-    fullk = api.VerifyDistill(d["D"], d["T"], head=head, draft_tok=draft, mode=w.mode,
-                              temperature=w.tau, seed=w.philox_seed, lam=w.lam, clip_c=w.clip_c,
-                              ws=ws, full_k=True, labels=True)
-    for _ in range(3):
-        fullk()
-    torch.cuda.synchronize()
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    n_fk = 20
-    f0.record(stream)
-    for _ in range(n_fk):
-        fullk()
-    f1.record(stream)
-    torch.cuda.synchronize()
-    fullk_ms = f0.elapsed_time(f1) / n_fk
-    fullk_bytes = algorithmic_bytes(np.full(w.B, w.k, np.int64), w.k, w.kt, w.V)
-    del fullk
-
-    # ---------------------------------------------------------------- vocab-sharded variant
-    vshard = None
-    if not args.no_vocab_shard and info.world == 1:
-        vshard = time_vocab_shard(w, d, bk, bk_host, draft, 8, stream)
-
     # ---------------------------------------------------------------- roofline of the row pass
     rows_avg_ms = statistics.mean(rows_ms)
     alg = algorithmic_bytes(bk_host, w.k, w.kt, w.V)
     achieved = alg / (rows_avg_ms / 1000.0) / 1e9
     peak, peak_kind = measured_peak()
-    traffic = recorded_traffic(args.workload)
+    traffic = recorded_traffic(w.name)
+    n_bonus = int((bk_host < w.kt).sum())
+
+    extra = {}
+    if headline:
+        # ------------------------------------------------------------ length-head online update
+        trainer = api.LengthHeadTrainer(d["W1"], d["b1"], d["w2"], d["b2"], w.B)
+        label = (fused.accept_len.float() / bk.float()).contiguous()   # the proxy label a / b_k
+        for _ in range(3):
+            trainer.step(d["h"], label)
+        torch.cuda.synchronize()
+        u0 = torch.cuda.Event(enable_timing=True)
+        u1 = torch.cuda.Event(enable_timing=True)
+        n_upd = 50
+        u0.record(stream)
+        for _ in range(n_upd):
+            trainer.step(d["h"], label)
+        u1.record(stream)
+        torch.cuda.synchronize()
+        extra["length_head_update_ms"] = u0.elapsed_time(u1) / n_upd
+
+        # ------------------------------------------------------------ full-k label mode
+        # the same step verifying and distilling all k rows (labels a/b_k and a/k both observable)
+        fullk = api.VerifyDistill(d["D"], d["T"], head=head, draft_tok=draft, mode=w.mode,
+                                  temperature=w.tau, seed=w.philox_seed, lam=w.lam, clip_c=w.clip_c,
+                                  ws=ws, full_k=True, labels=True)
+        for _ in range(3):
+            fullk()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        n_fk = 20
+        f0.record(stream)
+        for _ in range(n_fk):
+            fullk()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        fullk_ms = f0.elapsed_time(f1) / n_fk
+        fullk_bytes = algorithmic_bytes(np.full(w.B, w.k, np.int64), w.k, w.kt, w.V)
+        extra["full_k_step_ms"] = fullk_ms
+        extra["full_k_step_hbm_gbs"] = fullk_bytes / (fullk_ms / 1000.0) / 1e9
+        del fullk
+        # ------------------------------------------------------------ vocab-sharded variant
+        if not args.no_vocab_shard and info.world == 1:
+            extra["vocab_sharded"] = time_vocab_shard(w, d, bk, bk_host, draft, 8, stream)
+
+    # ---------------------------------------------------------------- (c, lambda) sweep
+    sweep_out = None
+    if sweep:
+        sweep_out = []
+        for c_, lam_ in sweep:
+            for v_ in (fused, rows_only):
+                v_.args.clip_c, v_.args.lambda_ = float(c_), float(lam_)
+            for _ in range(3):
+                fused()
+            n_sw = min(K, 20)
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(n_sw):
+                fused()
+            s1.record(stream)
+            r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            r0.record(stream)
+            for _ in range(n_sw):
+                rows_only()
+            r1.record(stream)
+            torch.cuda.synchronize()
+            if api.svd_get_device_error(ws) != 0:
+                raise SystemExit("device error in the sweep (%s)" % w.name)
+            rms = r0.elapsed_time(r1) / n_sw
+            sweep_out.append({"clip_c": None if math.isinf(c_) else c_, "lambda": lam_,
+                              "ms_per_step": s0.elapsed_time(s1) / n_sw, "row_pass_ms": rms,
+                              "frac": alg / (rms / 1000.0) / 1e9 / peak})
+        for v_ in (fused, rows_only):
+            v_.args.clip_c, v_.args.lambda_ = float(w.clip_c), float(w.lam)
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -478,6 +569,9 @@ def main():
                                  ("n_emitted", vd.n_emitted), ("loss_total", vd.loss_total),
                                  ("bk", bk))}
         h2d = host["D"].numel() * 2 + host["T"].numel() * 2 + host["h"].numel() * 2
+        if draft_host is not None:
+            draft_pin = draft_host.pin_memory()
+            h2d += draft_pin.numel() * 4
         d2h = sum(t.numel() * t.element_size() for t in out_host.values())
         if info.world > 1:
             torch.distributed.barrier()
@@ -489,6 +583,8 @@ def main():
             d["D"].copy_(host["D"], non_blocking=True)
             d["T"].copy_(host["T"], non_blocking=True)
             d["h"].copy_(host["h"], non_blocking=True)
+            if draft_host is not None:
+                draft.copy_(draft_pin, non_blocking=True)
             vd()
             for n, t in (("accept_len", vd.accept_len), ("emitted", vd.emitted),
                          ("n_emitted", vd.n_emitted), ("loss_total", vd.loss_total), ("bk", bk)):
@@ -498,57 +594,85 @@ def main():
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
         red_e = parallel.reduce_metrics(e2e_ms, verified, accepted, emitted, loss, device=dev)
         e2e = {"value": red_e["verified"] / (red_e["ms"] / 1000.0), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "copied_back": "accept_len, emitted, n_emitted, loss_total, b_k; the gradient "
+                              "dlogits stays on the device for the drafter's backward"}
 
     # ---------------------------------------------------------------- CPU oracle baseline
-    cpu = None
+    cpu, cases = None, None
     if info.rank == 0 and not args.no_cpu_baseline and info.world == 1:
         threads = os.cpu_count() or 1
         nseq = args.cpu_seqs or max(4, min(w.B, 2 * threads))
-        v, extra = cpu_oracle_sample(wr, host, nseq, threads)
+        target = 10.0 if headline else 4.0
+        v, ex = cpu_oracle_sample(wr, host, nseq, threads, target, draft=draft_host, bk_gpu=bk_host)
+        cases = ex["cases"]
         cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": "first %d of %d sequences x %d passes, fp64 oracle a1-a5 with gradient, "
-                         "%.1f s" % (nseq, w.B, extra["reps"], extra["seconds"])}
+                         "%.1f s" % (nseq, w.B, ex["reps"], ex["seconds"])}
+        if headline:
+            # the same sample on one host thread
+            n1 = max(2, nseq // 8)
+            v1, ex1 = cpu_oracle_sample(wr, host, n1, 1, target, draft=draft_host)
+            cpu["single_thread"] = {"value": v1, "unit": UNIT, "cores": 1,
+                                    "sample": "first %d sequences x %d passes, %.1f s"
+                                              % (n1, ex1["reps"], ex1["seconds"])}
+            oracle_threads_reset(threads)
+    if cases is None:
+        cases = {}
+    cases["bk_near_integer"] = bk_near
 
-    if info.rank == 0:
-        bk_hist = np.bincount(bk_host, minlength=w.k + 1)[1:].tolist()
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": red["ms"], "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": args.workload, "B": w.B, "k": w.k, "kt": w.kt, "V": w.V, "H": w.H,
-                       "M": w.M, "mode": "stochastic" if w.mode == 1 else "greedy", "lambda": w.lam, "clip_c": w.clip_c,
-                       "storage": "bf16 logits / bf16 gradient, fp32 arithmetic",
-                       "l2": "inputs larger than L2 (%.2f GB of logits per step, no flush)"
-                             % ((host["D"].numel() + host["T"].numel()) * 2 / 1e9),
-                       "parallelism": "dp%d (independent batch per GPU)" % info.world},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "row_pass_kernel", "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": alg,
-                         "avg_launch_ms": rows_avg_ms},
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            # length head, row pass, finalize per step (+ the stochastic draw)
-            "gpu_launches": (4 if w.mode == 1 else 3) * K,
-            "clocks": clock_rec,
-            "accepted_tokens_per_s": red["accepted"] / (red["ms"] / 1000.0),
-            "emitted_tokens_per_s": red["emitted"] / (red["ms"] / 1000.0),
-            "step_hbm_gbs": (alg + head_bytes(w.B, w.H, w.M)) * info.world / (red["ms"] / 1000.0) / 1e9,
-            "length_head_avg_ms": statistics.mean(head_ms),
-            "length_head_update_ms": update_ms,
-            "full_k_step_ms": fullk_ms,
-            "full_k_step_hbm_gbs": fullk_bytes / (fullk_ms / 1000.0) / 1e9,
-            "bk_hist": bk_hist,
-            "boundary_cases": {"bk_near_integer": bk_near},
-            "vocab_sharded": vshard,
-            "speedup_report": {k_: (None if v_ != v_ else round(v_, 6)) for k_, v_ in report.items()
-                               if k_ != "alpha"},
-        }
-        print(json.dumps(line), flush=True)
-    if info.world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    bk_hist = np.bincount(bk_host, minlength=w.k + 1)[1:].tolist()
+    leg = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": red["ms"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "k": w.k, "kt": w.kt, "V": w.V, "H": w.H,
+                   "M": w.M, "mode": "stochastic" if w.mode == 1 else "greedy", "lambda": w.lam,
+                   "clip_c": w.clip_c, "tau": w.tau,
+                   "storage": "bf16 logits / bf16 gradient, fp32 arithmetic",
+                   "l2": "inputs larger than L2 (%.2f GB of logits per step, no flush)"
+                         % ((host["D"].numel() + host["T"].numel()) * 2 / 1e9),
+                   "parallelism": "dp%d (independent batch per GPU)" % info.world},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "row_pass_kernel", "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": alg,
+                     "bytes_breakdown": {"sum_bk": int(bk_host.sum()), "bonus_rows": n_bonus,
+                                         "read_bytes": int(bk_host.sum()) * 4 * w.V + n_bonus * 2 * w.V,
+                                         "write_bytes": w.B * w.k * 2 * w.V,
+                                         "output_bytes": w.B * 4 * (3 + w.k + 1 + w.k)},
+                     "avg_launch_ms": rows_avg_ms},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        # the row pass (with the length head inside) and the finalize pass per step, plus the
+        # stochastic draw
+        "gpu_launches": (3 if w.mode == 1 else 2) * K,
+        "clocks": clock_rec,
+        "accepted_tokens_per_s": red["accepted"] / (red["ms"] / 1000.0),
+        "emitted_tokens_per_s": red["emitted"] / (red["ms"] / 1000.0),
+        "step_hbm_gbs": (alg + head_bytes(w.B, w.H, w.M)) * info.world / (red["ms"] / 1000.0) / 1e9,
+        "length_head_avg_ms": statistics.mean(head_ms),
+        "bk_hist": bk_hist,
+        "speedup_report": {k_: (None if v_ != v_ else round(v_, 6)) for k_, v_ in report.items()
+                           if k_ != "alpha"},
+        "_cases": cases,
+    }
+    if sweep_out is not None:
+        leg["sweep"] = sweep_out
+    leg.update(extra)
+    if not headline:
+        # a leg is not a bench line of its own: keep the figures, drop the contract's constants
+        for key in ("metric", "unit", "n_gpus", "warmup", "higher_is_better", "scaling",
+                    "vs_baseline", "data", "clocks"):
+            leg.pop(key, None)
+    del fused, rows_only, d, host, ws
+    torch.cuda.empty_cache()
+    return leg
+
+
+def oracle_threads_reset(n: int) -> None:
+    import oracle
+    oracle.set_threads(n)
 
 
 if __name__ == "__main__":

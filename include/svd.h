@@ -198,22 +198,27 @@ svd_status svd_verify_distill(const svd_verify_distill_args* args, void* ws, siz
  *
  * Scratch: a file-scope device array of SVD_NOALLOC_SCRATCH_BYTES in the library, one per
  * device.  Nothing is allocated, by the library or by anything it calls.
- *   - Set-up: the first call on each device (with that device current; `stream` must belong
- *     to the current device) looks up the array's address and caches it.  Make that first
- *     call before any stream capture begins.
+ *   - Set-up: the first call in each CUDA context (the runtime's primary context of a device,
+ *     or a driver-API context the caller made current) looks up the array's address in that
+ *     context and caches it under the context's unique id; a context destroyed and created
+ *     again (cudaDeviceReset) is a new context and is looked up again.  `stream` must belong
+ *     to the current context.  Make the first call in a context before any stream capture
+ *     begins.
+ *   - Checks: every argument is checked before the scratch is touched; a rejected call
+ *     enqueues nothing.
  *   - Zeroing: every call clears the svd_workspace_bytes(B, k, kt, M) bytes it uses with one
  *     cudaMemsetAsync on `stream`, so nothing needs to start at zero and an earlier device
  *     error leaves nothing behind.
  *   - Size limit: calls whose svd_workspace_bytes(B, k, kt, M) exceeds
  *     SVD_NOALLOC_SCRATCH_BYTES return SVD_ERR_WORKSPACE before anything is launched.
- *   - Concurrency: all calls on one device share the one array.  Calls that overlap on the
+ *   - Concurrency: all calls in one context share the one array.  Calls that overlap on the
  *     GPU (different streams, or host threads enqueuing without ordering) race on it and give
  *     undefined results; order them on one stream or with events.
  *   - Device errors: if `status_out` (a caller-owned DEVICE pointer to one uint32_t) is not
  *     NULL, the call's device status word (SVD_OK, SVD_ERR_TOKEN_RANGE or SVD_ERR_TIMEOUT) is
- *     copied there on `stream` after the kernels.
- * Other return codes as for svd_verify_distill; SVD_ERR_UNSUPPORTED for a device ordinal
- * of 64 or more. */
+ *     copied there on `stream` after the kernels.  It is written only when the call returns
+ *     SVD_OK; after any other return code its contents are unchanged.
+ * Other return codes as for svd_verify_distill. */
 svd_status svd_verify_distill_noalloc(const svd_verify_distill_args* args, uint32_t* status_out,
                                       void* stream);
 

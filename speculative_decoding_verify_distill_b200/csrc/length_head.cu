@@ -18,6 +18,7 @@
 #include <cmath>
 
 #include "svd_device.cuh"
+#include "svd_head_unit.cuh"
 
 namespace svd {
 
@@ -319,6 +320,13 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_cluster_kernel(const 
     if (t == 0) p.tile_ticket[bt] = 0u;
 }
 
+// The head as independent work units (svd_head_unit.cuh), one CTA per unit: the same units the
+// fused verify-and-distill pass runs inside its row pass, so both give the same bhat and b_k.
+__global__ void __launch_bounds__(kWarps * 32) length_head_units_kernel(const HeadParams p) {
+    __shared__ int flag;
+    head_unit<8>(p, static_cast<int>(blockIdx.x), &flag, true);
+}
+
 int launch_length_head(const HeadParams& p, void* stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool cluster_form = (p.H % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.h) & 15) == 0) &&
@@ -328,26 +336,8 @@ int launch_length_head(const HeadParams& p, void* stream) {
         length_head_kernel<<<grid, kWarps * 32, 0, st>>>(p);
         return static_cast<int>(cudaGetLastError());
     }
-    HeadParams q = p;
-    q.ks = (((p.H + kHeadCl - 1) / kHeadCl) + 15) & ~15;   // K columns per rank, multiple of 16
-    cudaError_t err = cudaFuncSetAttribute(length_head_cluster_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(kHeadClSmem));
-    if (err != cudaSuccess) return static_cast<int>(err);
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kHeadCl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cfg.gridDim = dim3(kHeadCl, (p.B + kHeadTileB - 1) / kHeadTileB, (p.M + kHeadTileM - 1) / kHeadTileM);
-    cfg.blockDim = dim3(kWarps * 32, 1, 1);
-    cfg.dynamicSmemBytes = kHeadClSmem;
-    cfg.stream = st;
-    err = cudaLaunchKernelEx(&cfg, length_head_cluster_kernel, q);
-    return static_cast<int>(err);
+    length_head_units_kernel<<<head_units(p), kWarps * 32, 0, st>>>(p);
+    return static_cast<int>(cudaGetLastError());
 }
 
 // ------------------------------------------------------------------------------------------

@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(kFixThreads) sample_fix_kernel(const RowParams
     __shared__ unsigned long long cm[kFixMaxCluster][2];   // [rank][residual, p] masses
     __shared__ unsigned long long scan[kFixWarps];
     __shared__ int found;
+    // launched as a programmatic dependent of the finalize pass: wait for its accepted lengths
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const uint32_t rank = cluster_rank(), CL = cluster_size();
     const int b = static_cast<int>(cluster_id_x());
@@ -191,13 +193,17 @@ int launch_sample_fix(const RowParams& p, void* stream) {
     const int per = (p.V + cl - 1) / cl;
     const int slice = (per + 7) & ~7;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // a programmatic dependent of the finalize pass (its CTAs start while finalize runs and
+    // wait in griddepcontrol.wait): the launch latency overlaps the finalize pass
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cfg.gridDim = dim3(static_cast<unsigned>(p.B) * cl, 1, 1);
     cfg.blockDim = dim3(kFixThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;

@@ -9,8 +9,12 @@
 // brings its own, of a fixed maximum size, created with the library's device image.
 //
 // Nothing here allocates: no cudaMalloc / cudaFree, no allocating library.  The scratch is a
-// static __device__ array; its address is looked up once per device (cudaGetSymbolAddress with
-// that device current) under a lock and cached.  Each call clears the bytes it uses with one
+// static __device__ array.  Its device address belongs to the CUDA context that loaded the
+// library's device image, not to the device number: a caller on the driver API may run under a
+// context of its own, and a context destroyed and re-created (cudaDeviceReset) maps the array
+// again, possibly elsewhere.  So the address is looked up (cudaGetSymbolAddress, with that
+// context current) once per context, keyed by the context's unique id, under a lock, and
+// cached.  Every call first checks all arguments, then clears the bytes it uses with one
 // cudaMemsetAsync on the caller's stream, runs the same kernels as svd_verify_distill on that
 // scratch, and (optionally) copies the device status word to a caller-owned device location.
 #include <cuda_runtime.h>
@@ -30,23 +34,67 @@ static_assert(kScratchBytes == SVD_NOALLOC_SCRATCH_BYTES, "header and library ag
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_lock;
-void* g_scratch_ptr[kMaxDevices] = {};
+// Context ids come from the driver (cuCtxGetCurrent + cuCtxGetId, CUDA 12.0), reached through
+// the runtime's entry-point query so that the library does not link the driver library itself.
+using CtxGetCurrentFn = int (*)(void** ctx);
+using CtxGetIdFn = int (*)(void* ctx, unsigned long long* id);
 
-// Device address of g_scratch on the current device; looked up on the first call per device.
-svd_status scratch_for_current_device(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SVD_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return SVD_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> guard(g_setup_lock);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return SVD_ERR_CUDA;
-        if ((reinterpret_cast<uintptr_t>(p) & 255u) != 0) return SVD_ERR_ALIGNMENT;
-        g_scratch_ptr[dev] = p;
+struct CacheEntry {
+    unsigned long long ctx_id;   // 0: empty
+    void* ptr;
+};
+constexpr int kCacheEntries = 64;
+std::mutex g_setup_lock;
+CacheEntry g_cache[kCacheEntries] = {};
+int g_cache_next = 0;            // round-robin slot for a new context once the cache is full
+bool g_driver_tried = false;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// Unique id of the current context; 0 if no context is current yet on this thread (the runtime
+// binds its primary context on the first call that needs one) or the driver cannot say.  With
+// id 0 the address is looked up without caching it.
+unsigned long long current_context_id() {
+    if (!g_driver_tried) {
+        g_driver_tried = true;
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f);
     }
-    *out = g_scratch_ptr[dev];
+    if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+    void* ctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_get_current(&ctx) != 0 || ctx == nullptr) return 0;
+    if (g_ctx_get_id(ctx, &id) != 0) return 0;
+    return id;
+}
+
+// Device address of g_scratch in the current context: looked up once per context.
+svd_status scratch_for_current_context(void** out) {
+    std::lock_guard<std::mutex> guard(g_setup_lock);
+    const unsigned long long id = current_context_id();
+    if (id != 0) {
+        for (int e = 0; e < kCacheEntries; ++e) {
+            if (g_cache[e].ctx_id == id) {
+                *out = g_cache[e].ptr;
+                return SVD_OK;
+            }
+        }
+    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return SVD_ERR_CUDA;
+    if ((reinterpret_cast<uintptr_t>(p) & 255u) != 0) return SVD_ERR_ALIGNMENT;
+    if (id != 0) {
+        g_cache[g_cache_next] = CacheEntry{id, p};
+        g_cache_next = (g_cache_next + 1) % kCacheEntries;
+    }
+    *out = p;
     return SVD_OK;
 }
 
@@ -54,15 +102,15 @@ svd_status scratch_for_current_device(void** out) {
 
 extern "C" svd_status svd_verify_distill_noalloc(const svd_verify_distill_args* a,
                                                  uint32_t* status_out, void* stream) {
-    if (a == nullptr) return SVD_ERR_INVALID_ARG;
+    // every argument check first: a rejected call touches neither the scratch nor the device
+    svd_status s = svd::check_verify_distill_args(a);
+    if (s != SVD_OK || a->B == 0) return s;
     const int M = a->h != nullptr ? a->M : 0;
     const size_t need = svd_workspace_bytes(a->B, a->k, a->kt, M);
-    // need == 0: a shape svd_verify_distill rejects; B == 0: nothing to launch.  Both return
-    // before the workspace is touched, so no scratch is set up for them.
-    if (need == 0 || a->B == 0) return svd_verify_distill(a, nullptr, 0, stream);
+    if (need == 0) return SVD_ERR_INVALID_ARG;
     if (need > kScratchBytes) return SVD_ERR_WORKSPACE;
     void* ws = nullptr;
-    svd_status s = scratch_for_current_device(&ws);
+    s = scratch_for_current_context(&ws);
     if (s != SVD_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the kernels expect an all-zero workspace; clearing it here also drops a status word or

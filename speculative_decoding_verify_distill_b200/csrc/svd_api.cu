@@ -58,9 +58,9 @@ svd_status from_cuda(int err) { return err == 0 ? SVD_OK : SVD_ERR_CUDA; }
 // Bound on any device-side wait: 1 s of wall-clock time (a staging copy lands in microseconds).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
-svd_status run_head(const uint16_t* h, const uint16_t* W1, const float* b1, const uint16_t* w2,
-                    float b2, int B, int H, int M, int k, float gamma, svd_bk_round rnd,
-                    float* bhat_out, int32_t* bk_out, const WsPtrs& w, void* stream) {
+HeadParams head_params(const uint16_t* h, const uint16_t* W1, const float* b1, const uint16_t* w2,
+                       float b2, int B, int H, int M, int k, float gamma, svd_bk_round rnd,
+                       float* bhat_out, int32_t* bk_out, const WsPtrs& w) {
     HeadParams p;
     p.h = h; p.W1 = W1; p.b1 = b1; p.w2 = w2; p.b2 = b2;
     p.B = B; p.H = H; p.M = M; p.k = k;
@@ -70,6 +70,13 @@ svd_status run_head(const uint16_t* h, const uint16_t* W1, const float* b1, cons
     p.nsplit = head_nsplit(B, M);
     const int per = (H + p.nsplit - 1) / p.nsplit;
     p.ks = (per + 15) & ~15;
+    return p;
+}
+
+svd_status run_head(const uint16_t* h, const uint16_t* W1, const float* b1, const uint16_t* w2,
+                    float b2, int B, int H, int M, int k, float gamma, svd_bk_round rnd,
+                    float* bhat_out, int32_t* bk_out, const WsPtrs& w, void* stream) {
+    const HeadParams p = head_params(h, W1, b1, w2, b2, B, H, M, k, gamma, rnd, bhat_out, bk_out, w);
     return from_cuda(launch_length_head(p, stream));
 }
 
@@ -79,7 +86,7 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
                     void* dlogits, float* loss_rows, float* loss_total, int32_t* accept_len,
                     int32_t* emitted, int32_t* n_emitted, svd_row_info* row_info, const WsPtrs& w,
                     void* stream, int bk_const = 0, float* label_proxy = nullptr,
-                    float* label_full = nullptr) {
+                    float* label_full = nullptr, const HeadParams* head = nullptr) {
     RowParams p;
     std::memset(&p, 0, sizeof p);
     p.D = D; p.T = T; p.draft = draft; p.bk = bk;
@@ -102,12 +109,45 @@ svd_status run_rows(const uint16_t* D, const uint16_t* T, const int32_t* draft, 
     p.bk_trunc = bk;
     p.label_proxy = label_proxy;
     p.label_full = label_full;
+    p.head_fused = head != nullptr ? 1 : 0;
+    if (head) p.head = *head;
     return from_cuda(launch_row_pass(p, stream));
 }
 
 bool bad_float(float x) { return !std::isfinite(x); }
 
 }  // namespace
+
+namespace svd {
+
+// Every argument check of svd_verify_distill that needs no workspace, in one place, so that
+// callers which bring their own scratch can reject a call before touching it.
+svd_status check_verify_distill_args(const svd_verify_distill_args* a) {
+    if (!a) return SVD_ERR_INVALID_ARG;
+    svd_status s = check_shape(a->B, a->k, a->kt, a->V);
+    if (s != SVD_OK) return s;
+    if (a->mode != SVD_GREEDY && a->mode != SVD_STOCHASTIC) return SVD_ERR_INVALID_ARG;
+    if (bad_float(a->temperature) || !(a->temperature > 0.f)) return SVD_ERR_INVALID_ARG;
+    if (bad_float(a->lambda) || a->lambda < 0.f || a->lambda > 1.f) return SVD_ERR_INVALID_ARG;
+    if (std::isnan(a->clip_c) || a->clip_c < 0.f || bad_float(a->grad_scale)) return SVD_ERR_INVALID_ARG;
+    if (a->dlogits_fp32 != 0 && a->dlogits_fp32 != 1) return SVD_ERR_INVALID_ARG;
+    if (a->full_k != 0 && a->full_k != 1) return SVD_ERR_INVALID_ARG;
+    if (a->h != nullptr) {
+        if (a->H < 1 || a->M < 1 || !a->W1 || !a->w2) return SVD_ERR_INVALID_ARG;
+        if (a->rnd != SVD_BK_CEIL && a->rnd != SVD_BK_FLOOR) return SVD_ERR_INVALID_ARG;
+        if (bad_float(a->b2) || bad_float(a->gamma) || !(a->gamma > 0.f)) return SVD_ERR_INVALID_ARG;
+    } else if (!a->bk_in && a->B > 0) {
+        return SVD_ERR_INVALID_ARG;
+    }
+    if (a->B == 0) return SVD_OK;
+    if (!a->D || !a->T || !a->bk || !a->accept_len || !a->emitted || !a->n_emitted ||
+        !a->loss_total || !a->dlogits)
+        return SVD_ERR_INVALID_ARG;
+    if (a->mode == SVD_STOCHASTIC && !a->draft_tok) return SVD_ERR_INVALID_ARG;
+    return SVD_OK;
+}
+
+}  // namespace svd
 
 extern "C" {
 
@@ -180,34 +220,24 @@ svd_status svd_distill_loss_grad(const uint16_t* D, const uint16_t* T, const int
 
 svd_status svd_verify_distill(const svd_verify_distill_args* a, void* ws, size_t ws_bytes,
                               void* stream) {
-    if (!a) return SVD_ERR_INVALID_ARG;
-    svd_status s = check_shape(a->B, a->k, a->kt, a->V);
-    if (s != SVD_OK) return s;
-    if (a->mode != SVD_GREEDY && a->mode != SVD_STOCHASTIC) return SVD_ERR_INVALID_ARG;
-    if (bad_float(a->temperature) || !(a->temperature > 0.f)) return SVD_ERR_INVALID_ARG;
-    if (bad_float(a->lambda) || a->lambda < 0.f || a->lambda > 1.f) return SVD_ERR_INVALID_ARG;
-    if (std::isnan(a->clip_c) || a->clip_c < 0.f || bad_float(a->grad_scale)) return SVD_ERR_INVALID_ARG;
-    if (a->dlogits_fp32 != 0 && a->dlogits_fp32 != 1) return SVD_ERR_INVALID_ARG;
-    if (a->full_k != 0 && a->full_k != 1) return SVD_ERR_INVALID_ARG;
+    svd_status s = svd::check_verify_distill_args(a);
+    if (s != SVD_OK || a->B == 0) return s;
     const bool head = a->h != nullptr;
-    if (head) {
-        if (a->H < 1 || a->M < 1 || !a->W1 || !a->w2) return SVD_ERR_INVALID_ARG;
-        if (a->rnd != SVD_BK_CEIL && a->rnd != SVD_BK_FLOOR) return SVD_ERR_INVALID_ARG;
-        if (bad_float(a->b2) || bad_float(a->gamma) || !(a->gamma > 0.f)) return SVD_ERR_INVALID_ARG;
-    } else if (!a->bk_in && a->B > 0) {
-        return SVD_ERR_INVALID_ARG;
-    }
-    if (a->B == 0) return SVD_OK;
-    if (!a->D || !a->T || !a->bk || !a->accept_len || !a->emitted || !a->n_emitted ||
-        !a->loss_total || !a->dlogits)
-        return SVD_ERR_INVALID_ARG;
-    if (a->mode == SVD_STOCHASTIC && !a->draft_tok) return SVD_ERR_INVALID_ARG;
     const int M = head ? a->M : 0;
     s = check_ws(ws, ws_bytes, a->B, a->k, a->kt, M);
     if (s != SVD_OK) return s;
     const WsPtrs w = carve(ws, a->B, a->k, a->kt, M);
     const int32_t* bk = a->bk;
-    if (head) {
+    // The length head runs inside the row pass (one launch less on the critical path) when its
+    // operands suit the tensor-core fragments read straight from L2 and the batch keeps its
+    // lists in shared memory; otherwise it runs as its own kernel first.
+    const bool fuse_head = head && a->B <= kRowCompactMaxB && a->H % 16 == 0 && aligned16(a->h) &&
+                           aligned16(a->W1);
+    HeadParams hp;
+    if (fuse_head) {
+        hp = head_params(a->h, a->W1, a->b1, a->w2, a->b2, a->B, a->H, a->M, a->k, a->gamma,
+                         a->rnd, a->bhat, a->bk, w);
+    } else if (head) {
         s = run_head(a->h, a->W1, a->b1, a->w2, a->b2, a->B, a->H, a->M, a->k, a->gamma, a->rnd,
                      a->bhat, a->bk, w, stream);
         if (s != SVD_OK) return s;
@@ -221,7 +251,7 @@ svd_status svd_verify_distill(const svd_verify_distill_args* a, void* ws, size_t
                     a->seed, a->step, a->lambda, a->clip_c, a->grad_scale, a->dlogits_fp32,
                     a->dlogits, a->loss_rows, a->loss_total, a->accept_len, a->emitted,
                     a->n_emitted, a->row_info, w, stream, a->full_k ? a->k : 0, a->label_proxy,
-                    a->label_full);
+                    a->label_full, fuse_head ? &hp : nullptr);
 }
 
 svd_status svd_length_head_update(const svd_head_update_args* a, void* ws, size_t ws_bytes,
@@ -257,6 +287,7 @@ svd_status svd_length_head_update(const svd_head_update_args* a, void* ws, size_
     if (s != SVD_OK) return s;
     HeadUpdateParams p;
     p.h = a->h; p.label = a->label; p.bhat = a->bhat; p.u = u; p.e = e;
+    p.ticket = &w.hdr->update_ticket;
     p.B = a->B; p.H = a->H; p.M = a->M;
     p.W1m = a->W1m; p.b1 = a->b1; p.w2m = a->w2m; p.b2 = a->b2; p.W1 = a->W1; p.w2 = a->w2;
     p.mW1 = a->mW1; p.vW1 = a->vW1; p.mb1 = a->mb1; p.vb1 = a->vb1;

@@ -167,6 +167,13 @@ __device__ __forceinline__ uint32_t redux_min_u32(uint32_t v) {
     return r;
 }
 
+// Three-input maximum (sm_100a form of max.f32; same NaN rule as fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Packed pairs of fp32 (sm_100a f32x2 forms; each half rounds exactly like the scalar op).
 __device__ __forceinline__ unsigned long long f2_bits(float2 a) {
     return *reinterpret_cast<unsigned long long*>(&a);
@@ -233,6 +240,14 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Load with acquire semantics at GPU scope (pairs with a release by another CTA: a
+// __threadfence before the writer's atomic).
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 // Record the first device-side error in the workspace status word.

@@ -19,7 +19,11 @@ struct WsHeader {
     uint32_t loss_ticket;  // finalize pass: CTAs finished
     uint32_t item_ticket;  // row pass: next loaded row to hand out (reset by the finalize pass)
     uint32_t zero_ticket;  // row pass: next zero-gradient unit to hand out (reset likewise)
-    uint32_t pad[59];
+    uint32_t head_unit;    // row pass with the length head inside: next head unit to hand out
+    uint32_t head_done;    // ... and the 16-sequence tiles whose b_k are written (both reset
+                           // by the finalize pass)
+    uint32_t update_ticket;  // length-head update: backward CTAs finished
+    uint32_t pad[56];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte line");
 
@@ -54,14 +58,14 @@ __host__ __device__ inline WsLayout ws_layout(int B, int k, int kt, int M) {
     off = align256(off + sizeof(float) * (size_t)mt * (size_t)B);
     L.part = off;
     off = align256(off + sizeof(float) * (size_t)head_nsplit(B, M) * (size_t)B * (size_t)(M > 0 ? M : 0));
-    L.tile_ticket = off;
-    off = align256(off + sizeof(uint32_t) * (size_t)bt * (size_t)mt);
+    L.tile_ticket = off;   // output-tile tickets [bt * mt], then sequence-tile tickets [bt]
+    off = align256(off + sizeof(uint32_t) * ((size_t)bt * (size_t)mt + (size_t)bt));
     // length-head update: pre-activations W1 h + b1 and backward terms, [B, M] fp32 each
     const size_t bm = (size_t)B * (size_t)(M > 0 ? M : 0);
     L.u = off;
     off = align256(off + sizeof(float) * bm);
-    L.e = off;
-    off = align256(off + sizeof(float) * bm);
+    L.e = off;   // backward terms: the w2 and b1 gradients [2, M] (at least)
+    off = align256(off + sizeof(float) * (bm > 2 * (size_t)(M > 0 ? M : 0) ? bm : 2 * (size_t)(M > 0 ? M : 0)));
     L.total = off;
     return L;
 }
@@ -85,13 +89,18 @@ struct HeadParams {
     WsHeader* hdr;
     float* zpart;            // [ceil(M/64), B] per-tile logits
     float* part;             // [nsplit, B, M] split partials of W1 h
-    uint32_t* tile_ticket;   // [ceil(B/16) * ceil(M/64)]
+    uint32_t* tile_ticket;   // [ceil(B/16) * ceil(M/64)] + [ceil(B/16)]
     int nsplit, ks;          // K splits and columns per split
 };
 
 // ------------------------------------------------------------------------------------------
 // row pass (verify + distill)
 // ------------------------------------------------------------------------------------------
+// Batches up to this size keep b_k and the prefixes of loaded and zero-gradient rows per
+// sequence in the row pass's shared memory (compact lists handed out dynamically); the length
+// head runs inside the row pass only for such batches.
+constexpr int kRowCompactMaxB = 4096;
+
 enum : int {
     kFlagVerify = 1,
     kFlagDistill = 2,
@@ -126,6 +135,9 @@ struct RowParams {
     const int32_t* bk_trunc;     // the truncated choice of b_k, for the labels
     float* label_proxy;          // [B] or null
     float* label_full;           // [B] or null
+    // length head computed inside the row pass (b_k written to `bk` before rows past 0 start)
+    int head_fused;
+    HeadParams head;
 };
 
 // Launchers (return cudaError_t as int; 0 = success).
@@ -139,7 +151,8 @@ struct HeadUpdateParams {
     const float* label;
     const float* bhat;
     const float* u;          // [B, M] pre-activations of the forward
-    float* e;                // [B, M] dl/d(pre-activation)
+    float* e;                // workspace: [2, M] w2 and b1 gradients
+    uint32_t* ticket;        // backward CTAs finished (back to zero after the step)
     int B, H, M;
     float *W1m, *b1, *w2m, *b2;
     uint16_t *W1, *w2;
@@ -160,5 +173,8 @@ struct RowGeometry {
     size_t smem;   // dynamic shared memory per CTA
 };
 bool row_geometry(int V, RowGeometry* g);
+
+// Argument checks of svd_verify_distill that need no workspace (SVD_OK when the call may go on).
+svd_status check_verify_distill_args(const svd_verify_distill_args* a);
 
 }  // namespace svd

@@ -42,8 +42,12 @@
 
 #include <cmath>
 #include <cstdio>
+#include <mutex>
+#include <utility>
+#include <vector>
 
 #include "svd_device.cuh"
+#include "svd_head_unit.cuh"
 
 namespace svd {
 
@@ -90,7 +94,9 @@ struct Ctl {
     Pending pend;
     int wscan[NW];                  // prologue scan of the loaded-row counts
     int wscanz[NW];                 // ... and of the zero-gradient row counts
-    uint32_t first_item;            // rank 0: the cluster's first loaded item (packed)
+    uint32_t first_raw[2];          // rank 0: the cluster's first loaded-item ticket (and a spare)
+    int hunit, hflag;               // length head inside the pass: current unit, its ticket flag
+    int list_flag;                  // the head has finished: build the compact lists
     int zs;                         // zero phase: the CTA's next unit
     int zu[2];                      // zero unit written while exchange #1 of a row is in flight
 };
@@ -98,7 +104,10 @@ struct Ctl {
 // Batches up to this size keep b_k and the prefixes of loaded and zero-gradient rows per sequence
 // in shared memory (compact lists, handed out dynamically); larger batches walk the uncompacted
 // (sequence, row) slots in a fixed order.
-constexpr int kCompactMaxB = 4096;
+constexpr int kCompactMaxB = kRowCompactMaxB;
+#ifndef SVD_HEAD_BATCH
+#define SVD_HEAD_BATCH 4
+#endif
 // Zero-gradient rows are handed out in sixteenths (about 19 KB of bf16 stores at V = 151936):
 // one unit per CTA fills the wait for each row's exchange, the rest follow the loaded rows.
 constexpr int kZeroSplit = 16;
@@ -152,7 +161,9 @@ __device__ __forceinline__ int first_zero_row(int n, bool verify) { return verif
 
 // Rows sequence b verifies: all k in full-k mode, else its b_k (clamped).
 __device__ __forceinline__ int load_bk(const RowParams& p, int b) {
-    return p.bk_const > 0 ? p.bk_const : clamp_bk(p, __ldg(p.bk + b));
+    if (p.bk_const > 0) return p.bk_const;
+    // b_k written by this grid's own head units is read through L2, not the read-only path
+    return clamp_bk(p, p.head_fused ? __ldcg(p.bk + b) : __ldg(p.bk + b));
 }
 // b_k of sequence b: from shared memory (compact mode) or global memory.
 struct BkView {
@@ -162,20 +173,24 @@ struct BkView {
     }
 };
 
-// Loaded item w of the whole batch.  Compact mode: w indexes the list of loaded rows ordered by
-// sequence (prefix sums in shared memory, binary search).  Otherwise w is a (sequence, row) slot
-// and holes decode to kItemNone.
-__device__ __forceinline__ Item decode_loaded(const RowParams& p, const int* spre, const BkView& bkv,
-                                              int w, bool verify) {
+// Loaded item w of the whole batch.  Compact mode: items 0 .. B-1 are row 0 of sequences
+// 0 .. B-1, which every sequence verifies whatever its b_k (b_k >= 1), so they need no b_k;
+// items from B on are the remaining loaded rows of each sequence in order (rows 1 .. b_k - 1 and
+// the bonus row), from the prefix sums spre of (loaded rows - 1) per sequence (binary search).
+// Otherwise w is a (sequence, row) slot and holes decode to kItemNone.
+__device__ __forceinline__ Item decode_loaded(const RowParams& p, bool compact, const int* spre,
+                                              const BkView& bkv, int w, bool verify) {
     Item it{kItemNone, -1, -1};
-    if (spre) {
-        if (w >= spre[p.B]) return it;
-        int lo = 0, hi = p.B;  // largest b with spre[b] <= w
+    if (compact) {
+        if (w < p.B) return Item{kItemRow, w, 0};
+        const int r = w - p.B;
+        if (r >= spre[p.B]) return it;
+        int lo = 0, hi = p.B;  // largest b with spre[b] <= r
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (spre[mid] <= w) lo = mid; else hi = mid;
+            if (spre[mid] <= r) lo = mid; else hi = mid;
         }
-        const int i = w - spre[lo];
+        const int i = 1 + (r - spre[lo]);
         const int n = bkv(p, lo);
         it = Item{i < n ? kItemRow : kItemBonus, lo, i};
     } else {
@@ -188,10 +203,6 @@ __device__ __forceinline__ Item decode_loaded(const RowParams& p, const int* spr
     return it;
 }
 
-// Number of loaded-item slots to walk (compact: exact count; otherwise all slots).
-__device__ __forceinline__ int loaded_slots(const RowParams& p, const int* spre) {
-    return spre ? spre[p.B] : p.B * p.kt;
-}
 
 
 }  // namespace
@@ -247,7 +258,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         mbar_init(&c.x2, 1);
         fence_mbar_init();
         c.my_ce[0] = c.my_ce[1] = 0.f;
-        c.first_item = 0u;
+        c.first_raw[0] = c.first_raw[1] = 0u;
     }
     // Vectors past the end of a warp's run hold a finite sentinel (the most negative bf16) in
     // both D and T: its exp is 0 and D - T is 0, so the passes run straight-line code over all
@@ -261,15 +272,16 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     }
     __syncthreads();
     const bool compact = p.B <= kCompactMaxB;
-    if (compact) {
-        // b_k and the exclusive prefixes of loaded rows and zero-gradient rows per sequence
+    // b_k and the exclusive prefixes of loaded rows past row 0 and of zero-gradient rows per
+    // sequence, in shared memory (the whole CTA takes part).
+    auto build_list = [&]() {
         int carry = 0, carryz = 0;
         for (int c0 = 0; c0 < p.B; c0 += NT) {
             const int b = c0 + t;
             int n = 0, L = 0, Z = 0;
             if (b < p.B) {
                 n = load_bk(p, b);
-                L = loaded_rows(n, kt, verify);
+                L = loaded_rows(n, kt, verify) - 1;
                 Z = DISTILL ? zero_rows(k, n, verify) : 0;
                 sbk[b] = n;
             }
@@ -300,25 +312,30 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         if (t == 0) {
             spre[p.B] = carry;
             zpre[p.B] = carryz;
-            // rank 0 takes the cluster's first loaded item from the workspace ticket
-            if (rank == 0) {
-                const int w0 = static_cast<int>(atomicAdd(&p.hdr->item_ticket, 1u));
-                c.first_item = pack_item(decode_loaded(p, spre, BkView{sbk}, w0, verify));
-            }
         }
+        __syncthreads();
+    };
+    // With the length head inside this pass, the lists wait for its b_k (full-k mode verifies
+    // every row and needs none).  Rows 0 need no list.
+    const bool head_first = p.head_fused && p.bk_const == 0;
+    bool list_ready = false;
+    if (compact && !head_first) {
+        build_list();
+        list_ready = true;
     }
+    // rank 0 takes the cluster's first loaded-item ticket
+    if (compact && rank == 0 && t == 0) c.first_raw[0] = atomicAdd(&p.hdr->item_ticket, 1u);
     __syncthreads();
-    cluster_sync();  // barriers, lists and the first item ready everywhere
+    cluster_sync();  // barriers, lists and the first ticket ready everywhere
 
     const BkView bkv{compact ? sbk : nullptr};
-    const int* list = compact ? spre : nullptr;
-    const int nslots = loaded_slots(p, list);
+    const int nslots = p.B * p.kt;   // (sequence, row) slots of the uncompacted walk
     // Compact mode: rank 0 takes loaded items one at a time from the workspace ticket, one row
     // ahead, and passes each in its exchange message.  Otherwise the cluster's items are slots
     // cid, cid + ncl, ...; holes are skipped.
     auto next_loaded = [&](int& w) -> Item {
         while (w < nslots) {
-            const Item it = decode_loaded(p, list, bkv, w, verify);
+            const Item it = decode_loaded(p, false, nullptr, bkv, w, verify);
             if (it.kind != kItemNone) return it;
             w += ncl;
         }
@@ -371,7 +388,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     };
 
     // unit u of the compact zero-row list: a sixteenth of gradient row (b, i), i past b_k
-    const int zunits = (DISTILL && compact) ? zpre[p.B] * kZeroSplit : 0;
+    int zunits = (DISTILL && compact && list_ready) ? zpre[p.B] * kZeroSplit : 0;
     auto write_zero_unit = [&](int u) {
         const int j = u / kZeroSplit, qq = u % kZeroSplit;
         int lo = 0, hi = p.B;  // largest b with zpre[b] <= j
@@ -400,16 +417,73 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         }
     };
 
+    // Thread 0: whether the length head has written every b_k; with `block`, waits for it at most
+    // the wait limit.  A wait that runs out records a timeout, and the lists are then built from
+    // b_k as they stand (every value is clamped to [1, k], so no access leaves its row).
+    auto head_finished = [&](bool block) -> bool {
+        const uint32_t need = static_cast<uint32_t>(head_seq_tiles(p.head));
+        if (ld_acquire_gpu(&p.hdr->head_done) >= need) return true;
+        if (!block) return false;
+        const uint64_t t0 = global_timer_ns();
+        while (ld_acquire_gpu(&p.hdr->head_done) < need) {
+            if (global_timer_ns() - t0 > p.wait_limit_ns) {
+                set_device_error(&p.hdr->status, SVD_ERR_TIMEOUT);
+                return true;
+            }
+            __nanosleep(256);
+        }
+        return true;
+    };
+    // The whole CTA: build the lists if the head has finished (with `block` from thread 0: once
+    // it has).
+    auto try_list = [&](bool block) {
+        if (t == 0) c.list_flag = head_finished(block) ? 1 : 0;
+        __syncthreads();
+        if (c.list_flag) {
+            build_list();
+            list_ready = true;
+            zunits = DISTILL ? zpre[p.B] * kZeroSplit : 0;
+        }
+    };
+
     Item cur{kItemNone, -1, -1};
     int w = cid;
+    int raw0 = 0;
+    bool cur_issued = false;
     if (compact) {
         uint32_t v = 0;
-        if (lane == 0) v = dsmem_ld_u32(dsmem_map(&c.first_item, 0));
-        cur = unpack_item(__shfl_sync(0xffffffffu, v, 0));
+        if (lane == 0) v = dsmem_ld_u32(dsmem_map(&c.first_raw[0], 0));
+        raw0 = static_cast<int>(__shfl_sync(0xffffffffu, v, 0));
+        // a row-0 item (or any item, once the lists exist) starts loading right away
+        if (raw0 < p.B || list_ready) {
+            cur = decode_loaded(p, true, spre, bkv, raw0, verify);
+            if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
+            cur_issued = true;
+        }
     } else {
         cur = next_loaded(w);
+        if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
+        cur_issued = true;
     }
-    if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
+    // The length head's work units, taken from a ticket by whichever CTAs are running (no unit
+    // waits for another, so the head finishes even if only part of the grid is resident), while
+    // the first row's copies land.
+    if (p.head_fused) {
+        const int U = head_units(p.head);
+        while (true) {
+            if (t == 0) c.hunit = static_cast<int>(atomicAdd(&p.hdr->head_unit, 1u));
+            __syncthreads();
+            const int u = c.hunit;
+            __syncthreads();
+            if (u >= U) break;
+            head_unit<SVD_HEAD_BATCH>(p.head, u, &c.hflag, false);
+        }
+    }
+    if (compact && !cur_issued) {
+        if (!list_ready) try_list(true);
+        cur = decode_loaded(p, true, spre, bkv, raw0, verify);
+        if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
+    }
     uint32_t phase = 0;          // parity of this warp's staging barrier
     bool wait_dead = false;      // a bounded wait ran out: skip later waits so the kernel ends
     int it = 0;                  // loaded rows done (row parity selects the exchange #1 buffers)
@@ -464,6 +538,9 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         // rank 0 asks for the next item now; it travels in this row's message #1
         uint32_t fetched = 0;
         if (compact && rank == 0 && t == 0) fetched = atomicAdd(&p.hdr->item_ticket, 1u);
+        // until the head has finished: build the lists as soon as it has, and before rank 0
+        // decodes a ticket past the row-0 items
+        if (compact && !list_ready) try_list(rank == 0 && fetched >= static_cast<uint32_t>(p.B));
         // and every CTA asks for one zero-row unit to write while this row's exchange is in flight
         int zfetch = 0;
         if (zunits > 0 && t == 0) zfetch = static_cast<int>(atomicAdd(&p.hdr->zero_ticket, 1u));
@@ -592,8 +669,8 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
                 aDd = fma2(ed[2], dd[2], aDd);
                 aDd = fma2(ed[3], dd[3], aDd);
                 if (DISTILL) {
-                    dmax = fmaxf(dmax, fmaxf(fmaxf(fmaxf(dd[0].x, dd[0].y), fmaxf(dd[1].x, dd[1].y)),
-                                             fmaxf(fmaxf(dd[2].x, dd[2].y), fmaxf(dd[3].x, dd[3].y))));
+                    dmax = fmax3(fmax3(dd[0].x, dd[0].y, dd[1].x), fmax3(dd[1].y, dd[2].x, dd[2].y),
+                                 fmax3(dd[3].x, dd[3].y, dmax));
                 }
             }
         }
@@ -643,7 +720,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             uint32_t nitem = 0u;
             if (compact && rank == 0) {
                 const int fw = static_cast<int>(__shfl_sync(0xffffffffu, fetched, 0));
-                nitem = pack_item(decode_loaded(p, list, bkv, fw, verify));
+                nitem = pack_item(decode_loaded(p, true, spre, bkv, fw, verify));
             }
             // the previous row's -log q_y (if this CTA owns its y) goes out with this row's message
             const float pce = c.my_ce[par ^ 1];
@@ -916,6 +993,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
 
     // ---------------------------------------------------------------- zero-only gradient rows
     if (DISTILL && compact) {
+        if (!list_ready) try_list(true);
         // the zero-row units not yet taken, handed to CTAs one at a time (the next unit is
         // requested while the current one is written)
         const int units = zunits;
@@ -962,15 +1040,20 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
 // ------------------------------------------------------------------------------------------
 // finalize: per sequence, the acceptance scan over its row records (one lane per position),
 // the emitted tokens, the loss rows past b_k and the sequence loss; the last CTA adds the
-// sequence losses in sequence order.
+// sequence losses in a fixed order (per lane in sequence order, then a butterfly).
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) finalize_kernel(const RowParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the stochastic draw (a programmatic dependent of this pass) may be scheduled now; it waits
+    // for this grid's results
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ int last;
     // the row pass has finished: its work tickets go back to zero for the next call
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         p.hdr->item_ticket = 0u;
         p.hdr->zero_ticket = 0u;
+        p.hdr->head_unit = 0u;
+        p.hdr->head_done = 0u;
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool verify = (p.flags & kFlagVerify) != 0;
@@ -1042,7 +1125,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(const RowParams p) {
         }
     }
     if (!distill) return;
-    // the last CTA adds the sequence losses in sequence order
+    // the last CTA adds the sequence losses in a fixed order
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -1050,12 +1133,17 @@ __global__ void __launch_bounds__(256) finalize_kernel(const RowParams p) {
         last = (old + 1u == gridDim.x) ? 1 : 0;
     }
     __syncthreads();
-    if (!last || threadIdx.x != 0) return;
+    if (!last || threadIdx.x >= 32) return;
     __threadfence();
+    // warp 0: lane l adds sequences l, l + 32, ... in order, then a fixed butterfly
     float tot = 0.f;
-    for (int s = 0; s < p.B; ++s) tot += __ldcg(p.seq_loss + s);
-    *p.loss_total = tot;
-    p.hdr->loss_ticket = 0u;
+#pragma unroll 4
+    for (int s = lane; s < p.B; s += 32) tot += __ldcg(p.seq_loss + s);
+    tot = warp_sum(tot);
+    if (lane == 0) {
+        *p.loss_total = tot;
+        p.hdr->loss_ticket = 0u;
+    }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1130,6 +1218,62 @@ size_t row_smem_bytes(const RowGeometry& g, int B) {
     return g.smem + list;
 }
 
+namespace {
+
+// Resident clusters of a row-pass kernel on the current device, for a launch with `smem` bytes of
+// dynamic shared memory.  The function attributes are set once per (device, kernel) -- to the
+// largest dynamic shared memory any batch size can ask for -- and the occupancy query once per
+// (device, kernel, smem); both under a lock, so concurrent first calls from several host
+// threads neither race on the cache nor on the attributes.
+struct OccEntry {
+    int dev;
+    KernelFn fn;
+    size_t smem;
+    int clusters;
+};
+std::mutex g_occ_lock;
+std::vector<OccEntry> g_occ;                     // occupancy per (device, kernel, smem)
+std::vector<std::pair<int, KernelFn>> g_attr;    // (device, kernel) with attributes set
+
+int resident_clusters(KernelFn fn, const RowGeometry& geo, size_t smem, cudaLaunchConfig_t cfg,
+                      int* out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return static_cast<int>(err);
+    std::lock_guard<std::mutex> guard(g_occ_lock);
+    for (const OccEntry& e : g_occ) {
+        if (e.dev == dev && e.fn == fn && e.smem == smem) {
+            *out = e.clusters;
+            return 0;
+        }
+    }
+    bool attr_set = false;
+    for (const auto& a : g_attr) attr_set = attr_set || (a.first == dev && a.second == fn);
+    if (!attr_set) {
+        err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(row_smem_bytes(geo, kCompactMaxB)));
+        if (err != cudaSuccess) return static_cast<int>(err);
+        // the same kernel serves vocabularies whose clusters exceed the portable size of 8
+        err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (err != cudaSuccess) return static_cast<int>(err);
+        g_attr.emplace_back(dev, fn);
+    }
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cfg.gridDim = dim3(geo.cluster * sms, 1, 1);
+    int n = 0;
+    err = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
+    if (err != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = sms / geo.cluster > 0 ? sms / geo.cluster : 1;
+    }
+    g_occ.push_back(OccEntry{dev, fn, smem, n});
+    *out = n;
+    return 0;
+}
+
+}  // namespace
+
 int launch_row_pass(const RowParams& p, void* stream) {
     RowGeometry geo;
     if (!row_geometry(p.V, &geo)) return static_cast<int>(cudaErrorInvalidValue);
@@ -1138,13 +1282,6 @@ int launch_row_pass(const RowParams& p, void* stream) {
                 : geo.variant == 1 ? pick_kernel<kLNT, kLNV, kLMB>(p.flags, aligned)
                                    : pick_kernel<kXNT, kXNV, kXMB>(p.flags, aligned);
     const size_t smem = row_smem_bytes(geo, p.B);
-    cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-    if (err != cudaSuccess) return static_cast<int>(err);
-    if (geo.cluster > 8) {
-        err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (err != cudaSuccess) return static_cast<int>(err);
-    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1156,25 +1293,10 @@ int launch_row_pass(const RowParams& p, void* stream) {
     cfg.blockDim = dim3(geo.threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    // persistent grid: as many clusters as can be resident at once (cached per configuration)
-    static int cached_clusters[3][17][8][2] = {};
-    static size_t cached_smem[3][17][8][2] = {};
-    int& cache = cached_clusters[geo.variant][geo.cluster][p.flags & 7][aligned ? 1 : 0];
-    size_t& csm = cached_smem[geo.variant][geo.cluster][p.flags & 7][aligned ? 1 : 0];
-    if (cache == 0 || csm != smem) {
-        int dev = 0, sms = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cfg.gridDim = dim3(geo.cluster * sms, 1, 1);
-        int n = 0;
-        err = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
-        if (err != cudaSuccess || n < 1) {
-            cudaGetLastError();
-            n = sms / geo.cluster > 0 ? sms / geo.cluster : 1;
-        }
-        cache = n;
-        csm = smem;
-    }
+    // persistent grid: as many clusters as can be resident at once
+    int cache = 0;
+    cudaError_t err = static_cast<cudaError_t>(resident_clusters(fn, geo, smem, cfg, &cache));
+    if (err != cudaSuccess) return static_cast<int>(err);
     const long long max_items = static_cast<long long>(p.B) * (p.kt + p.k);
     int nclusters = cache;
     if (max_items < nclusters) nclusters = static_cast<int>(max_items > 0 ? max_items : 1);

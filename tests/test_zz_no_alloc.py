@@ -26,7 +26,8 @@ def L():
 
 
 def test_rejections_before_any_launch(L):
-    """Argument and size errors return before the scratch is set up (no CUDA call is made)."""
+    """Argument and size errors return before the scratch is set up (no CUDA call is made):
+    every argument check runs first, then the size check."""
     assert L.svd_verify_distill_noalloc(None, None, None) == 1
     fake = ctypes.c_void_p(0x1000)   # never dereferenced
     a = api.VerifyDistillArgs()
@@ -42,6 +43,16 @@ def test_rejections_before_any_launch(L):
     assert L.svd_verify_distill_noalloc(ctypes.byref(a), None, None) == 1
     a.k = 16
     assert L.svd_verify_distill_noalloc(ctypes.byref(a), None, None) == 0   # empty batch
+    # bad arguments on a shape too large for the scratch: the argument error wins, because
+    # every argument is checked before the size, the scratch or the stream is touched
+    a.B = 20000
+    for field, bad in (("mode", 7), ("temperature", float("nan")), ("k", 33), ("kt", 18),
+                       ("lambda_", 1.5), ("clip_c", -1.0), ("full_k", 2)):
+        good = getattr(a, field)
+        setattr(a, field, bad)
+        assert L.svd_verify_distill_noalloc(ctypes.byref(a), None, None) == 1, field
+        setattr(a, field, good)
+    assert L.svd_verify_distill_noalloc(ctypes.byref(a), None, None) == 3
 
 
 def _snapshot(vd):
