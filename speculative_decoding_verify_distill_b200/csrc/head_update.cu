@@ -10,11 +10,13 @@
 //
 // Kernels: the forward, with its pre-activations stored, is the length-head kernel; the whole
 // backward and the AdamW steps are one kernel (head_back_kernel below): dl/dW1 = E^T h
-// ([M,B] x [B,H], 0.27 GFLOP at B=128, H=4096, M=256) on fp32 CUDA cores with shared-memory
-// tiles, each output summed over b in order, with E formed on the fly from the stored
-// pre-activations; the w2, b1, b2 gradients and their AdamW steps in the last CTA.  fp32
-// throughout: Adam's first step is lr * g / |g|, so the sign of small gradients matters, and the
-// contraction is too small for tensor-core tiles to pay.
+// ([M,B] x [B,H], 0.27 GFLOP at B=128, H=4096, M=256) on the tensor cores (mma.sync m16n8k16,
+// fp32 accumulation), with E formed on the fly from the stored pre-activations and fed as the
+// sum of three bf16 operands (hi = RN(e), mid = RN(e - hi), lo = RN(e - hi - mid): e h to
+// within 2^-24 relative, since h is exact in bf16); the w2, b1, b2 gradients and their AdamW
+// steps in the last CTA.  Accuracy
+// matters here because Adam's first step is lr * g / |g|: the sign of a small gradient decides
+// the direction of the step.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -54,23 +56,40 @@ __device__ __forceinline__ float delta_of(const HeadUpdateParams& p, int b) {
 // One kernel for the whole backward.  CTA (jt, mt) owns the 64 x 64 block of W1 (units
 // m0 .. m0 + 63, hidden columns j0 .. j0 + 63).  Per chunk of 64 sequences it forms
 // e_bm = delta_b w2_m [u_bm > 0] for its units in shared memory (from the forward's stored
-// pre-activations u, so no separate pass writes e), stages the matching h columns, and adds
-// e_bm h_bj into its 4 x 4 outputs per thread, sequences in order.  The AdamW step on its block
-// of W1 follows (16-byte loads and stores).  The CTAs of column 0 also sum the w2 and b1
+// pre-activations u, so no separate pass writes e), stages the matching h columns, and its
+// eight warps add E^T h into four 16 x 8 tiles each on the tensor cores.  The AdamW step on its
+// block of W1 follows (8-byte loads and stores).  The CTAs of column 0 also sum the w2 and b1
 // gradients of their units over the sequences (four threads per unit, combined in order) into
 // the workspace; the last CTA to finish (atomic ticket) applies AdamW to w2, b1 and b2 and forms
 // the loss -- only then, because every CTA reads the forward's w2 to form e.
 constexpr int kBC = 64;          // sequences per chunk
 constexpr int kHLd = kTile + 8;  // bf16 row pitch of the staged h tile (16-byte rows)
+constexpr int kELd = kTile + 4;  // fp32 row pitch of the e tile (fragment reads on distinct banks)
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               const uint32_t (&b)[2]) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// Two fp32 to bf16 with round-to-nearest-even, the first in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
 
 __global__ void __launch_bounds__(256) head_back_kernel(const HeadUpdateParams p) {
-    __shared__ __align__(16) float se[kBC][kTile];        // e[b0 + r, m0 + c]
+    __shared__ __align__(16) float se[kBC][kELd];         // e[b0 + r, m0 + c]
     __shared__ __align__(16) uint16_t sh[kBC][kHLd];      // h[b0 + r, j0 + c]
     __shared__ float sdelta[kBC];
     __shared__ float sg[2][4][kTile];                     // w2 / b1 gradient partials
     __shared__ int last;
-    const int t = threadIdx.x;
-    const int tx = t & 15, ty = t >> 4;         // outputs (m0 + 4ty + i, j0 + 4tx + jj)
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    // tensor-core tiles: warp w owns hidden units m0 + 16 (w & 3) .. + 15 and columns
+    // j0 + 32 (w >> 2) .. + 31, i.e. four 16 x 8 output tiles
+    const int g = lane >> 2, tq = lane & 3;
+    const int mb = (warp & 3) * 16, jb = (warp >> 2) * 32;
     const int j0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile;
     const bool col0 = blockIdx.x == 0;
     // e-tile role: unit c = t % 64, rows r = t / 64, t / 64 + 4, ...
@@ -79,7 +98,7 @@ __global__ void __launch_bounds__(256) head_back_kernel(const HeadUpdateParams p
     const float w2f = ulive ? bf16_to_f32(__ldg(p.w2 + m0 + ec)) : 0.f;   // the forward's weight
     const bool hvec = (p.H % 8 == 0) && ((reinterpret_cast<uintptr_t>(p.h) & 15) == 0) && (j0 + kTile <= p.H);
     float gw = 0.f, gb = 0.f;
-    float acc[4][4];
+    float acc[4][4];   // [tile nt][(g, 2tq), (g, 2tq + 1), (g + 8, 2tq), (g + 8, 2tq + 1)]
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -133,54 +152,78 @@ __global__ void __launch_bounds__(256) head_back_kernel(const HeadUpdateParams p
             }
         }
         __syncthreads();
-        for (int r = 0; r < nb; ++r) {   // sequences in order
-            const float4 e4 = *reinterpret_cast<const float4*>(&se[r][4 * ty]);
-            const uint2 h4 = *reinterpret_cast<const uint2*>(&sh[r][4 * tx]);
-            const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
-            const float hv[4] = {__uint_as_float(h4.x << 16), __uint_as_float(h4.x & 0xffff0000u),
-                                 __uint_as_float(h4.y << 16), __uint_as_float(h4.y & 0xffff0000u)};
+        // dW1 tile += E^T h over the chunk's sequences, 16 at a time, on the tensor cores
+        // (mma.sync m16n8k16, fp32 accumulation).  E is fp32: it enters as the sum of three
+        // bf16 operands, hi = RN(e), mid = RN(e - hi), lo = RN(e - hi - mid), whose products
+        // with the exact bf16 h add up to e h within 2^-24 relative, as fine as e itself;
+        // rows past the batch hold zeros.
+        for (int kb = 0; kb < nb; kb += 16) {
+            uint32_t ahi[4], amid[4], alo[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int q = 0; q < 4; ++q) {
+                // a0: (row g, k 2tq..2tq+1), a1: row g + 8, a2: k + 8, a3: both
+                const int m = mb + g + ((q & 1) ? 8 : 0);
+                const int r = kb + 2 * tq + ((q & 2) ? 8 : 0);
+                const float e0 = se[r][m], e1 = se[r + 1][m];
+                const uint32_t hi = pack_bf16x2_rn(e0, e1);
+                const float r0 = e0 - __uint_as_float(hi << 16), r1 = e1 - __uint_as_float(hi & 0xffff0000u);
+                const uint32_t mid = pack_bf16x2_rn(r0, r1);
+                ahi[q] = hi;
+                amid[q] = mid;
+                alo[q] = pack_bf16x2_rn(r0 - __uint_as_float(mid << 16), r1 - __uint_as_float(mid & 0xffff0000u));
+            }
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(ev[i], hv[jj], acc[i][jj]);
+            for (int nt = 0; nt < 4; ++nt) {
+                const int j = jb + nt * 8 + g;
+                const int r = kb + 2 * tq;
+                uint32_t bf[2];
+                bf[0] = static_cast<uint32_t>(sh[r][j]) | (static_cast<uint32_t>(sh[r + 1][j]) << 16);
+                bf[1] = static_cast<uint32_t>(sh[r + 8][j]) | (static_cast<uint32_t>(sh[r + 9][j]) << 16);
+                // smallest part first, so the larger parts are added to an accumulator that
+                // already holds the small corrections
+                mma_bf16_16816(acc[nt], alo, bf);
+                mma_bf16_16816(acc[nt], amid, bf);
+                mma_bf16_16816(acc[nt], ahi, bf);
+            }
         }
         __syncthreads();
     }
-    // AdamW epilogue on this thread's 4 x 4 block of W1: every master weight and moment is
-    // loaded before the first store
-    const bool wvec = (p.H % 4 == 0) && (j0 + 4 * tx + 4 <= p.H) &&
+    // AdamW epilogue on this lane's entries of W1: (m, j .. j + 1) for the rows g and g + 8 of
+    // each of its four tiles; masters and moments with 8-byte loads and stores
+    const bool wvec = (p.H % 2 == 0) &&
                       (((reinterpret_cast<uintptr_t>(p.W1m) | reinterpret_cast<uintptr_t>(p.mW1) |
-                         reinterpret_cast<uintptr_t>(p.vW1)) & 15) == 0) &&
-                      ((reinterpret_cast<uintptr_t>(p.W1) & 7) == 0);
+                         reinterpret_cast<uintptr_t>(p.vW1)) & 7) == 0) &&
+                      ((reinterpret_cast<uintptr_t>(p.W1) & 3) == 0);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int m = m0 + 4 * ty + i;
-        if (m >= p.M) continue;
-        const size_t o = static_cast<size_t>(m) * p.H + j0 + 4 * tx;
-        if (wvec) {
-            float4 wm = *reinterpret_cast<const float4*>(p.W1m + o);
-            float4 mm = *reinterpret_cast<const float4*>(p.mW1 + o);
-            float4 vv = *reinterpret_cast<const float4*>(p.vW1 + o);
-            float w[4] = {wm.x, wm.y, wm.z, wm.w}, m1[4] = {mm.x, mm.y, mm.z, mm.w},
-                  v1[4] = {vv.x, vv.y, vv.z, vv.w};
+    for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) w[jj] = adamw(w[jj], acc[i][jj], m1[jj], v1[jj], p);
-            *reinterpret_cast<float4*>(p.W1m + o) = make_float4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<float4*>(p.mW1 + o) = make_float4(m1[0], m1[1], m1[2], m1[3]);
-            *reinterpret_cast<float4*>(p.vW1 + o) = make_float4(v1[0], v1[1], v1[2], v1[3]);
-            const uint2 wb = make_uint2(f32_to_bf16_rne(w[0]) | (uint32_t(f32_to_bf16_rne(w[1])) << 16),
-                                        f32_to_bf16_rne(w[2]) | (uint32_t(f32_to_bf16_rne(w[3])) << 16));
-            *reinterpret_cast<uint2*>(p.W1 + o) = wb;
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                if (j0 + 4 * tx + jj >= p.H) continue;
-                float mm = p.mW1[o + jj], vv = p.vW1[o + jj];
-                const float w = adamw(p.W1m[o + jj], acc[i][jj], mm, vv, p);
-                p.W1m[o + jj] = w;
-                p.mW1[o + jj] = mm;
-                p.vW1[o + jj] = vv;
-                p.W1[o + jj] = f32_to_bf16_rne(w);
+        for (int half = 0; half < 2; ++half) {
+            const int m = m0 + mb + g + 8 * half;
+            const int j = j0 + jb + nt * 8 + 2 * tq;
+            if (m >= p.M || j >= p.H) continue;
+            const size_t o = static_cast<size_t>(m) * p.H + j;
+            const float g0 = acc[nt][2 * half], g1 = acc[nt][2 * half + 1];
+            if (wvec && j + 1 < p.H) {
+                const float2 wm = *reinterpret_cast<const float2*>(p.W1m + o);
+                float2 mm = *reinterpret_cast<const float2*>(p.mW1 + o);
+                float2 vv = *reinterpret_cast<const float2*>(p.vW1 + o);
+                const float w0 = adamw(wm.x, g0, mm.x, vv.x, p);
+                const float w1 = adamw(wm.y, g1, mm.y, vv.y, p);
+                *reinterpret_cast<float2*>(p.W1m + o) = make_float2(w0, w1);
+                *reinterpret_cast<float2*>(p.mW1 + o) = mm;
+                *reinterpret_cast<float2*>(p.vW1 + o) = vv;
+                *reinterpret_cast<uint32_t*>(p.W1 + o) =
+                    f32_to_bf16_rne(w0) | (static_cast<uint32_t>(f32_to_bf16_rne(w1)) << 16);
+            } else {
+                const float gg[2] = {g0, g1};
+                for (int jj = 0; jj < 2 && j + jj < p.H; ++jj) {
+                    float mm = p.mW1[o + jj], vv = p.vW1[o + jj];
+                    const float w = adamw(p.W1m[o + jj], gg[jj], mm, vv, p);
+                    p.W1m[o + jj] = w;
+                    p.mW1[o + jj] = mm;
+                    p.vW1[o + jj] = vv;
+                    p.W1[o + jj] = f32_to_bf16_rne(w);
+                }
             }
         }
     }
@@ -220,20 +263,28 @@ __global__ void __launch_bounds__(256) head_back_kernel(const HeadUpdateParams p
         p.mb1[m] = mm;
         p.vb1[m] = vv;
     }
-    if (t == 0) {
-        // loss and b2 gradient over the sequences in order
+    if (t < 32) {
+        // loss and b2 gradient: lane l adds sequences l, l + 32, ... in order, then a butterfly
         float ls = 0.f, gs = 0.f;
-        for (int b = 0; b < p.B; ++b) {
+#pragma unroll 4
+        for (int b = t; b < p.B; b += 32) {
             const float e = __ldg(p.bhat + b) - __ldg(p.label + b);
             ls += e * e;
             gs += delta_of(p, b);
         }
-        *p.loss = ls / static_cast<float>(p.B);
-        float mm = *p.mb2, vv = *p.vb2;
-        *p.b2 = adamw(*p.b2, gs, mm, vv, p);
-        *p.mb2 = mm;
-        *p.vb2 = vv;
-        *p.ticket = 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            gs += __shfl_xor_sync(0xffffffffu, gs, o);
+        }
+        if (t == 0) {
+            *p.loss = ls / static_cast<float>(p.B);
+            float mm = *p.mb2, vv = *p.vb2;
+            *p.b2 = adamw(*p.b2, gs, mm, vv, p);
+            *p.mb2 = mm;
+            *p.vb2 = vv;
+            *p.ticket = 0u;
+        }
     }
 }
 

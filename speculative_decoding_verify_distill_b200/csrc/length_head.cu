@@ -322,9 +322,25 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_cluster_kernel(const 
 
 // The head as independent work units (svd_head_unit.cuh), one CTA per unit: the same units the
 // fused verify-and-distill pass runs inside its row pass, so both give the same bhat and b_k.
-__global__ void __launch_bounds__(kWarps * 32) length_head_units_kernel(const HeadParams p) {
+// Dynamic shared memory: the unit's staged K chunk, then its mbarrier.
+__global__ void __launch_bounds__(kWarps * 32) length_head_units_kernel(const HeadParams p,
+                                                                       uint32_t stage_bytes) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + stage_bytes);
     __shared__ int flag;
-    head_unit<8>(p, static_cast<int>(blockIdx.x), &flag, true);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    uint32_t phase = 0;
+    head_unit<kWarps>(p, static_cast<int>(blockIdx.x), &flag, true, reinterpret_cast<uint16_t*>(smem_raw),
+                      stage_bytes, bar, phase, kHeadWaitNs);
+}
+
+// Shared memory for a unit whose split of ks columns is staged in one chunk.
+size_t head_unit_stage_bytes(int ks) {
+    return static_cast<size_t>(kHeadTileB + kHeadTileM) * (ks + 8) * 2;
 }
 
 int launch_length_head(const HeadParams& p, void* stream) {
@@ -336,7 +352,16 @@ int launch_length_head(const HeadParams& p, void* stream) {
         length_head_kernel<<<grid, kWarps * 32, 0, st>>>(p);
         return static_cast<int>(cudaGetLastError());
     }
-    length_head_units_kernel<<<head_units(p), kWarps * 32, 0, st>>>(p);
+    // one chunk per unit when it fits in 100 KB, else chunks of what does
+    size_t stage = head_unit_stage_bytes(p.ks);
+    if (stage > 100 * 1024) stage = 100 * 1024;
+    stage = (stage + 127) & ~size_t(127);
+    const size_t smem = stage + 16;
+    cudaError_t err = cudaFuncSetAttribute(length_head_units_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return static_cast<int>(err);
+    length_head_units_kernel<<<head_units(p), kWarps * 32, smem, st>>>(p, static_cast<uint32_t>(stage));
     return static_cast<int>(cudaGetLastError());
 }
 

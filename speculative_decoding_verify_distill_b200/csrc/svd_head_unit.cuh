@@ -10,9 +10,10 @@
 //     b_k = clamp(round(gamma * bhat_b * k), 1, k)   (round = ceil or floor).
 //
 // Work units: (16-sequence tile bt) x (64-unit tile mt) x (K split kz).  A unit is one CTA (any
-// multiple of 32 threads, at least 32): its warps take the eight 16 x 8 blocks of hidden units
-// m0 + 8j .. m0 + 8j + 7 in turn and accumulate each over the split's K range on the tensor cores (mma.sync m16n8k16, bf16 operands read straight from L2
-// into fragments, fp32 accumulation) and stores it as a split partial.  The last unit of an
+// multiple of 32 threads, at least 32): it stages its slices of h and W1 in shared memory with
+// bulk copies, its warps take the eight 16 x 8 blocks of hidden units in turn and accumulate each
+// over the split's K range on the tensor cores (mma.sync m16n8k16, bf16 operands, fp32
+// accumulation), and the unit stores its block as a split partial.  The last unit of an
 // output tile (atomic ticket, no waiting) adds the partials in split order, applies b1, ReLU and
 // w2 and sums the tile's 64 units per sequence; the last tile of a sequence tile adds the tile
 // sums in tile order and applies the sigmoid and the b_k map, then counts the sequence tile as
@@ -42,15 +43,31 @@ __host__ __device__ inline int head_seq_tiles(const HeadParams& p) {
     return (p.B + kHeadTileB - 1) / kHeadTileB;
 }
 
-// One unit, executed by all threads of the calling CTA (H a multiple of 16; h, W1 4-byte
-// aligned rows).  `flag` is one int of the CTA's shared memory.  The tickets live in
-// p.tile_ticket: [bt * mt] output-tile tickets, then [bt] sequence-tile tickets; every ticket is
-// back at zero once its last user has finished.  p.hdr->head_done counts finished sequence tiles.
-// kBatch k-steps of fragments are in flight at a time (registers: 6 per k-step).
-// With `standalone` (a kernel that only runs the head), the last sequence tile also puts
-// head_done back to zero; inside the row pass the finalize pass does, after the rows have read it.
-template <int kBatch>
-__device__ __forceinline__ void head_unit(const HeadParams& p, int u, int* flag, bool standalone) {
+// Columns of one staged K chunk that fit in `smem_bytes` of shared memory: 16 rows of h and 64
+// rows of W1, each padded by 8 bf16 (16 bytes) so that fragment reads hit distinct banks.
+__host__ __device__ inline int head_chunk_cols(size_t smem_bytes) {
+    const long cols = static_cast<long>(smem_bytes / (2 * (kHeadTileB + kHeadTileM))) - 8;
+    return cols < 16 ? 0 : static_cast<int>(cols & ~15L);
+}
+
+// One unit, executed by all threads of the calling CTA (H a multiple of 16; h and W1 16-byte
+// aligned).  The split's K range is staged in chunks: one bulk copy (1-D TMA, no multicast) per
+// row of h and of W1 into `stage` (smem_bytes of this CTA's shared memory), completing on the
+// mbarrier `bar` (count 1; `phase` is its parity, flipped per chunk), then the warps take the
+// eight 16 x 8 blocks of hidden units m0 + 8j .. m0 + 8j + 7 in turn and accumulate them over
+// the chunk from shared memory.  A chunk costs one round trip to memory.  `flag` is one int of
+// the CTA's shared memory.  The tickets live in p.tile_ticket: [bt * mt] output-tile tickets,
+// then [bt] sequence-tile tickets; every ticket is back at zero once its last user has
+// finished.  p.hdr->head_done counts finished sequence tiles.  With `standalone` (a kernel that
+// only runs the head), the last sequence tile also puts head_done back to zero; inside the row
+// pass the finalize pass does, after the rows have read it.  Returns false if a staging wait
+// ran out (the status word then says SVD_ERR_TIMEOUT).
+template <int NW>
+__device__ __forceinline__ bool head_unit(const HeadParams& p, int u, int* flag, bool standalone,
+                                          uint16_t* stage, size_t smem_bytes, uint64_t* bar,
+                                          uint32_t& phase, uint64_t wait_limit_ns) {
+    constexpr int nw = NW;                          // warps of the calling CTA
+    constexpr int kPer = (kHeadTileM / 8 + NW - 1) / NW;   // 16 x 8 blocks per warp
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int BT = (p.B + kHeadTileB - 1) / kHeadTileB, MT = (p.M + kHeadTileM - 1) / kHeadTileM;
     const int kz = u % p.nsplit;
@@ -59,36 +76,65 @@ __device__ __forceinline__ void head_unit(const HeadParams& p, int u, int* flag,
     const int b0 = bt * kHeadTileB, m0 = mt * kHeadTileM;
     const int g = lane >> 2, tq = lane & 3;
     const int k_lo = min(p.H, kz * p.ks), k_hi = min(p.H, k_lo + p.ks);
+    const int nrow_h = min(kHeadTileB, p.B - b0), nrow_w = min(kHeadTileM, p.M - m0);
+    const int cmax = head_chunk_cols(smem_bytes);
+    const int nchunk = k_hi > k_lo ? (k_hi - k_lo + cmax - 1) / cmax : 0;
+    const int cw = nchunk > 0 ? (((k_hi - k_lo + nchunk - 1) / nchunk) + 15) & ~15 : 0;
+    const int ld = cw + 8;                              // row pitch in bf16
+    uint16_t* hs = stage;
+    uint16_t* ws = stage + kHeadTileB * ld;
+    bool ok = true;
 
-    // ------------------------------------------------ split partials, one 16 x 8 block per warp
-    const int nw = static_cast<int>(blockDim.x >> 5);
-    for (int blk = warp; blk < kHeadTileM / 8; blk += nw) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const int r0 = b0 + g, r1 = b0 + g + 8, mrow = m0 + blk * 8 + g;
-        const uint32_t* h0 = r0 < p.B ? reinterpret_cast<const uint32_t*>(p.h + static_cast<size_t>(r0) * p.H) : nullptr;
-        const uint32_t* h1 = r1 < p.B ? reinterpret_cast<const uint32_t*>(p.h + static_cast<size_t>(r1) * p.H) : nullptr;
-        const uint32_t* wr = mrow < p.M ? reinterpret_cast<const uint32_t*>(p.W1 + static_cast<size_t>(mrow) * p.H) : nullptr;
-        // fragments of kBatch k-steps are loaded before any of their products, so each batch
-        // costs one L2 round trip rather than one per k-step
-        for (int kb = k_lo; kb < k_hi; kb += 16 * kBatch) {
-            uint32_t a[kBatch][4], bf[kBatch][2];
+    // ------------------------------------------------ split partials, 16 x 8 blocks by warp
+    // (a warp owns blocks warp, warp + nw, ...)
+    float acc[kPer][4];
 #pragma unroll
-            for (int s = 0; s < kBatch; ++s) {
-                const int kk = kb + 16 * s;
-                const bool in = kk < k_hi;
-                const int c = (kk >> 1) + tq;      // 32-bit word index of columns kk + 2 tq
-                a[s][0] = (in && h0) ? __ldg(h0 + c) : 0u;
-                a[s][1] = (in && h1) ? __ldg(h1 + c) : 0u;
-                a[s][2] = (in && h0) ? __ldg(h0 + c + 4) : 0u;
-                a[s][3] = (in && h1) ? __ldg(h1 + c + 4) : 0u;
-                bf[s][0] = (in && wr) ? __ldg(wr + c) : 0u;
-                bf[s][1] = (in && wr) ? __ldg(wr + c + 4) : 0u;
-            }
+    for (int j = 0; j < kPer; ++j)
 #pragma unroll
-            for (int s = 0; s < kBatch; ++s)
-                if (kb + 16 * s < k_hi) mma_16816_bf16(acc, a[s], bf[s]);
+        for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
+    // rows past the batch or the hidden size read as zeros
+    for (int x = t; x < (kHeadTileB - nrow_h) * ld; x += blockDim.x) hs[nrow_h * ld + x] = 0;
+    for (int x = t; x < (kHeadTileM - nrow_w) * ld; x += blockDim.x) ws[nrow_w * ld + x] = 0;
+    for (int ch = 0; ch < nchunk; ++ch) {
+        const int c0 = k_lo + ch * cw, c1 = min(k_hi, c0 + cw);
+        __syncthreads();      // every read of the previous chunk (and the zero rows) is done
+        if (t == 0) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            const uint32_t row_bytes = static_cast<uint32_t>(c1 - c0) * 2u;
+            mbar_arrive_expect_tx(bar, row_bytes * static_cast<uint32_t>(nrow_h + nrow_w));
+            for (int r = 0; r < nrow_h; ++r)
+                bulk_load(hs + r * ld, p.h + static_cast<size_t>(b0 + r) * p.H + c0, row_bytes, bar);
+            for (int r = 0; r < nrow_w; ++r)
+                bulk_load(ws + r * ld, p.W1 + static_cast<size_t>(m0 + r) * p.H + c0, row_bytes, bar);
         }
-        // accumulator layout: acc[0..1] = (row g, cols 2tq + {0,1}); acc[2..3] = row g + 8
+        if (ok && !mbar_wait_bounded(bar, phase, wait_limit_ns)) {
+            ok = false;
+            set_device_error(&p.hdr->status, SVD_ERR_TIMEOUT);
+        }
+        phase ^= 1u;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int blk = warp + j * nw;
+            if (blk >= kHeadTileM / 8) break;
+            const uint16_t* wrow = ws + (blk * 8 + g) * ld;
+            for (int kk = 0; kk < c1 - c0; kk += 16) {
+                uint32_t a[4], bf[2];
+                a[0] = *reinterpret_cast<const uint32_t*>(hs + g * ld + kk + 2 * tq);
+                a[1] = *reinterpret_cast<const uint32_t*>(hs + (g + 8) * ld + kk + 2 * tq);
+                a[2] = *reinterpret_cast<const uint32_t*>(hs + g * ld + kk + 2 * tq + 8);
+                a[3] = *reinterpret_cast<const uint32_t*>(hs + (g + 8) * ld + kk + 2 * tq + 8);
+                bf[0] = *reinterpret_cast<const uint32_t*>(wrow + kk + 2 * tq);
+                bf[1] = *reinterpret_cast<const uint32_t*>(wrow + kk + 2 * tq + 8);
+                mma_16816_bf16(acc[j], a, bf);
+            }
+        }
+    }
+    __syncthreads();          // the staging area is free again when this returns
+    // accumulator layout: acc[j][0..1] = (row g, cols 2tq + {0,1}); acc[j][2..3] = row g + 8
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int blk = warp + j * nw;
+        if (blk >= kHeadTileM / 8) break;
         float* part = p.part + static_cast<size_t>(kz) * p.B * p.M;
         const int m = m0 + blk * 8 + 2 * tq;
         const int rows[2] = {b0 + g, b0 + g + 8};
@@ -96,8 +142,8 @@ __device__ __forceinline__ void head_unit(const HeadParams& p, int u, int* flag,
         for (int h2 = 0; h2 < 2; ++h2) {
             const int b = rows[h2];
             if (b < p.B) {
-                if (m < p.M) part[static_cast<size_t>(b) * p.M + m] = acc[2 * h2];
-                if (m + 1 < p.M) part[static_cast<size_t>(b) * p.M + m + 1] = acc[2 * h2 + 1];
+                if (m < p.M) part[static_cast<size_t>(b) * p.M + m] = acc[j][2 * h2];
+                if (m + 1 < p.M) part[static_cast<size_t>(b) * p.M + m + 1] = acc[j][2 * h2 + 1];
             }
         }
     }
@@ -109,7 +155,7 @@ __device__ __forceinline__ void head_unit(const HeadParams& p, int u, int* flag,
         *flag = (old + 1u == static_cast<uint32_t>(p.nsplit)) ? 1 : 0;
     }
     __syncthreads();
-    if (!*flag) return;
+    if (!*flag) return ok;
     __threadfence();
     // one warp per row of the tile; lane: units lane and lane + 32 (fixed orders)
     for (int r = warp; r < kHeadTileB; r += nw) {
@@ -149,7 +195,7 @@ __device__ __forceinline__ void head_unit(const HeadParams& p, int u, int* flag,
         *flag = (old + 1u == static_cast<uint32_t>(MT)) ? 2 : 0;
     }
     __syncthreads();
-    if (*flag != 2) return;
+    if (*flag != 2) return ok;
     __threadfence();
     if (t < kHeadTileB && b0 + t < p.B) {
         const int b = b0 + t;
@@ -178,6 +224,7 @@ __device__ __forceinline__ void head_unit(const HeadParams& p, int u, int* flag,
         const uint32_t old = atomicAdd(&p.hdr->head_done, 1u);
         if (standalone && old + 1u == static_cast<uint32_t>(BT)) p.hdr->head_done = 0u;
     }
+    return ok;
 }
 
 }  // namespace svd

@@ -70,7 +70,7 @@ struct alignas(16) Msg1 {          // after pass A
     uint32_t argT, argD;            // lowest id holding mT / mD in the sender's slice
     float prev_ce;                  // -log q_y of the previous row from the owner of y, else 0
     uint32_t next_item;             // rank 0: the cluster's next loaded item (packed)
-    uint32_t pad0, pad1;
+    float Dx, Tx;                   // stochastic: D and T at the draft token from its owner, else 0
 };
 struct alignas(16) Msg2 {          // after pass B: clipped reverse-KL entries
     float clip_d, clip_q, n_clip, pad0;
@@ -90,6 +90,7 @@ struct Ctl {
     Msg1 in1[2][16];                // exchange #1 by row parity and sender rank
     Msg2 in2[16];                   // exchange #2 by sender rank
     uint64_t x1[2], x2;             // exchange barriers
+    uint64_t hbar;                  // length head inside the pass: its staging barrier
     float my_ce[2];                 // -log q_y computed in this CTA, by row parity
     Pending pend;
     int wscan[NW];                  // prologue scan of the loaded-row counts
@@ -105,9 +106,7 @@ struct Ctl {
 // in shared memory (compact lists, handed out dynamically); larger batches walk the uncompacted
 // (sequence, row) slots in a fixed order.
 constexpr int kCompactMaxB = kRowCompactMaxB;
-#ifndef SVD_HEAD_BATCH
-#define SVD_HEAD_BATCH 4
-#endif
+
 // Zero-gradient rows are handed out in sixteenths (about 19 KB of bf16 stores at V = 151936):
 // one unit per CTA fills the wait for each row's exchange, the rest follow the loaded rows.
 constexpr int kZeroSplit = 16;
@@ -132,7 +131,7 @@ __device__ __forceinline__ Msg1 empty_msg1() {
     m.argT = m.argD = kNone;
     m.prev_ce = 0.f;
     m.next_item = 0u;
-    m.pad0 = m.pad1 = 0u;
+    m.Dx = m.Tx = 0.f;
     return m;
 }
 
@@ -256,20 +255,24 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         mbar_init(&c.x1[0], 1);
         mbar_init(&c.x1[1], 1);
         mbar_init(&c.x2, 1);
+        mbar_init(&c.hbar, 1);
         fence_mbar_init();
         c.my_ce[0] = c.my_ce[1] = 0.f;
         c.first_raw[0] = c.first_raw[1] = 0u;
     }
     // Vectors past the end of a warp's run hold a finite sentinel (the most negative bf16) in
     // both D and T: its exp is 0 and D - T is 0, so the passes run straight-line code over all
-    // NV rounds with no per-vector branches.  The bulk copies never touch this tail.
-    {
+    // NV rounds with no per-vector branches.  The bulk copies never touch this tail.  (With the
+    // length head inside the pass, the staging area serves the head first; the tail is written
+    // after it.)
+    auto fill_sentinel = [&]() {
         const uint4 sent = make_uint4(0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu);
         for (int lv = wcnt + lane; lv < NV * 32; lv += 32) {
             myD[lv] = sent;
             myT[lv] = sent;
         }
-    }
+    };
+    if (!p.head_fused) fill_sentinel();
     __syncthreads();
     const bool compact = p.B <= kCompactMaxB;
     // b_k and the exclusive prefixes of loaded rows past row 0 and of zero-gradient rows per
@@ -446,46 +449,44 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         }
     };
 
-    Item cur{kItemNone, -1, -1};
-    int w = cid;
-    int raw0 = 0;
-    bool cur_issued = false;
-    if (compact) {
-        uint32_t v = 0;
-        if (lane == 0) v = dsmem_ld_u32(dsmem_map(&c.first_raw[0], 0));
-        raw0 = static_cast<int>(__shfl_sync(0xffffffffu, v, 0));
-        // a row-0 item (or any item, once the lists exist) starts loading right away
-        if (raw0 < p.B || list_ready) {
-            cur = decode_loaded(p, true, spre, bkv, raw0, verify);
-            if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
-            cur_issued = true;
-        }
-    } else {
-        cur = next_loaded(w);
-        if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
-        cur_issued = true;
-    }
+    bool wait_dead = false;      // a bounded wait ran out: skip later waits so the kernel ends
     // The length head's work units, taken from a ticket by whichever CTAs are running (no unit
-    // waits for another, so the head finishes even if only part of the grid is resident), while
-    // the first row's copies land.
+    // waits for another, so the head finishes even if only part of the grid is resident), staged
+    // through this CTA's (still idle) staging area before its first row uses it.
     if (p.head_fused) {
         const int U = head_units(p.head);
+        uint32_t hphase = 0;
         while (true) {
             if (t == 0) c.hunit = static_cast<int>(atomicAdd(&p.hdr->head_unit, 1u));
             __syncthreads();
             const int u = c.hunit;
             __syncthreads();
             if (u >= U) break;
-            head_unit<SVD_HEAD_BATCH>(p.head, u, &c.hflag, false);
+            if (!head_unit<NW>(p.head, u, &c.hflag, false, reinterpret_cast<uint16_t*>(stageD),
+                               static_cast<size_t>(NV) * NT * 32, &c.hbar, hphase, p.wait_limit_ns))
+                wait_dead = true;
         }
+        fill_sentinel();
+        __syncthreads();
     }
-    if (compact && !cur_issued) {
-        if (!list_ready) try_list(true);
+
+    Item cur{kItemNone, -1, -1};
+    int w = cid;
+    if (compact) {
+        uint32_t v = 0;
+        if (lane == 0) v = dsmem_ld_u32(dsmem_map(&c.first_raw[0], 0));
+        const int raw0 = static_cast<int>(__shfl_sync(0xffffffffu, v, 0));
+        // a row-0 item needs no list; a later one waits for the head's b_k
+        if (raw0 >= p.B && !list_ready) try_list(true);
         cur = decode_loaded(p, true, spre, bkv, raw0, verify);
-        if (ALIGNED && lane == 0 && cur.kind != kItemNone) issue_loads(cur);
+    } else {
+        cur = next_loaded(w);
+    }
+    if (ALIGNED && lane == 0 && cur.kind != kItemNone) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // after the head's reads
+        issue_loads(cur);
     }
     uint32_t phase = 0;          // parity of this warp's staging barrier
-    bool wait_dead = false;      // a bounded wait ran out: skip later waits so the kernel ends
     int it = 0;                  // loaded rows done (row parity selects the exchange #1 buffers)
     uint32_t n2 = 0;             // completed phases of exchange barrier #2
     bool pending = false;        // rank 0 owes the record of the previous loaded row
@@ -553,26 +554,13 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
         // exps are needed for distillation rows and for the stochastic ratio and sampler (lse)
         const bool need_lse = (DISTILL && isRow) || STOCH;
 
-        // caller's draft token and, in stochastic mode, D_x and T_x for the acceptance ratio
+        // The caller's draft token: loaded now, first used after pass A (its latency hides behind
+        // the staging wait and pass A).  In stochastic mode D_x and T_x come from the staged
+        // slice of the CTA that holds x, through the exchange: no dependent global loads.
         uint32_t x = kNone;
         float Dx = 0.f, Tx = 0.f;
-        if (rowVerify && p.draft != nullptr) {
-            int xv = 0;
-            if (lane == 0) {
-                xv = __ldg(p.draft + drow);
-                if (xv < 0 || xv >= V) {
-                    if (warp == 0) set_device_error(&p.hdr->status, SVD_ERR_TOKEN_RANGE);
-                    xv = -1;
-                } else if (STOCH) {
-                    Dx = __uint_as_float(static_cast<uint32_t>(__ldg(p.D + drow * V + xv)) << 16);
-                    Tx = __uint_as_float(static_cast<uint32_t>(__ldg(p.T + trow * V + xv)) << 16);
-                }
-            }
-            xv = __shfl_sync(0xffffffffu, xv, 0);
-            Dx = __shfl_sync(0xffffffffu, Dx, 0);
-            Tx = __shfl_sync(0xffffffffu, Tx, 0);
-            x = xv < 0 ? kNone : static_cast<uint32_t>(xv);
-        }
+        int xraw = -1;
+        if (rowVerify && p.draft != nullptr && lane == 0) xraw = __ldg(p.draft + drow);
 
         // -------------------------------------------------------- staging
         if (ALIGNED) {
@@ -675,6 +663,33 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             }
         }
 
+        // the caller's token, range-checked; the lane whose staged vector holds it reads D_x, T_x
+        float wDx = 0.f, wTx = 0.f;
+        if (rowVerify && p.draft != nullptr) {
+            int xv = __shfl_sync(0xffffffffu, xraw, 0);
+            if (xv < 0 || xv >= V) {
+                if (warp == 0 && lane == 0) set_device_error(&p.hdr->status, SVD_ERR_TOKEN_RANGE);
+                xv = -1;
+            }
+            x = xv < 0 ? kNone : static_cast<uint32_t>(xv);
+            if (STOCH && xv >= 0) {
+                const int xl = xv - v0;
+                float dv = 0.f, tv = 0.f;
+                if (xl >= 0 && xl < len) {
+                    const int vi = xl >> 3;
+                    if (vi / vpw == warp && ((vi - wv0) & 31) == lane) {
+                        const int lvx = vi - wv0;
+                        dv = __uint_as_float(static_cast<uint32_t>(
+                            reinterpret_cast<const uint16_t*>(myD + lvx)[xl & 7]) << 16);
+                        tv = __uint_as_float(static_cast<uint32_t>(
+                            reinterpret_cast<const uint16_t*>(myT + lvx)[xl & 7]) << 16);
+                    }
+                }
+                wDx = warp_sum(dv);    // one lane of the cluster holds them; the rest add zeros
+                wTx = warp_sum(tv);
+            }
+        }
+
         // warp partials -> shared memory -> warp 0 -> message #1 to every rank
         {
             const float wmD = redux_max_f32(RD), wmT = redux_max_f32(RT);
@@ -696,7 +711,8 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             }
             m.prev_ce = 0.f;
             m.next_item = 0u;
-            m.pad0 = m.pad1 = 0u;
+            m.Dx = wDx;
+            m.Tx = wTx;
             if (lane == 0) c.w1[warp] = m;
         }
         if (zunits > 0 && t == 0) c.zu[par] = zfetch;
@@ -707,6 +723,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             const uint32_t cargT = redux_min_u32(a.mT == cmT ? a.argT : kNone);
             const uint32_t cargD = redux_min_u32(a.mD == cmD ? a.argD : kNone);
             const float cdmax = redux_max_f32(a.dmax);
+            const float cDx = STOCH ? warp_sum(a.Dx) : 0.f, cTx = STOCH ? warp_sum(a.Tx) : 0.f;
             float csD = 0.f, csDd = 0.f, csT = 0.f;
             if (need_lse) {
                 const float fT = rescale(a.mT, cmT, k2);
@@ -726,7 +743,7 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             const float pce = c.my_ce[par ^ 1];
             send1(make_uint4(__float_as_uint(cmD), __float_as_uint(csD), __float_as_uint(csDd), __float_as_uint(cdmax)),
                   make_uint4(__float_as_uint(cmT), __float_as_uint(csT), cargT, cargD),
-                  make_uint4(__float_as_uint(pce), nitem, 0u, 0u), par);
+                  make_uint4(__float_as_uint(pce), nitem, __float_as_uint(cDx), __float_as_uint(cTx)), par);
             __syncwarp();
             if (lane == 0) c.my_ce[par ^ 1] = 0.f;
         }
@@ -745,6 +762,10 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
             MT = redux_max_f32(a.mT);
             y = redux_min_u32(a.mT == MT ? a.argT : kNone);
             if (greedy_x && isRow) x = redux_min_u32(a.mD == MD ? a.argD : kNone);
+            if (STOCH && rowVerify) {
+                Dx = warp_sum(a.Dx);
+                Tx = warp_sum(a.Tx);
+            }
             if (compact) nxt = unpack_item(__shfl_sync(0xffffffffu, a.next_item, 0));
             if (need_lse) {
                 const float sT = warp_sum(a.sT * rescale(a.mT, MT, k2));
