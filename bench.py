@@ -505,6 +505,24 @@ def run_leg(w, args, info, dev, *, headline: bool, sweep=None):
         u1.record(stream)
         torch.cuda.synchronize()
         extra["length_head_update_ms"] = u0.elapsed_time(u1) / n_upd
+        # the update right after a verification step on the same hidden states, reusing that
+        # step's head forward (its pre-activations and bhat): only the backward kernel runs
+        step_pre = api.VerifyDistill(d["D"], d["T"], head=trainer.head(d["h"]), draft_tok=draft,
+                                     mode=w.mode, temperature=w.tau, seed=w.philox_seed,
+                                     lam=w.lam, clip_c=w.clip_c, ws=ws, labels=True,
+                                     head_preact=True)
+        ev_u = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_upd)]
+        for j in range(n_upd + 3):
+            step_pre()
+            if j >= 3:
+                ev_u[j - 3][0].record(stream)
+            trainer.step(d["h"], step_pre.label_proxy, preact=step_pre.head_preact, bhat=step_pre.bhat)
+            if j >= 3:
+                ev_u[j - 3][1].record(stream)
+        torch.cuda.synchronize()
+        extra["length_head_update_after_step_ms"] = statistics.mean(
+            e[0].elapsed_time(e[1]) for e in ev_u)
+        del step_pre
 
         # ------------------------------------------------------------ full-k label mode
         # the same step verifying and distilling all k rows (labels a/b_k and a/k both observable)

@@ -178,6 +178,10 @@ typedef struct svd_verify_distill_args {
     float* label_proxy;      /* [B] or NULL: a / b_k as truncated verification observes it;
                               * with full_k = 1, min(a, b_k) / b_k                            */
     float* label_full;       /* [B] or NULL: a / k with full_k = 1; NaN with full_k = 0         */
+    /* [B,M] fp32 or NULL: the head's pre-activations W1 h + b1, written when the head runs.  With
+     * `bhat`, they are the forward an online update of the head on the same hidden states and
+     * served weights needs (svd_head_update_args.preact), so that update need not recompute it. */
+    float* head_preact;
 } svd_verify_distill_args;
 
 /* a1 .. a5 in one call: the length head (unless h == NULL), then one persistent pass over the
@@ -247,7 +251,13 @@ typedef struct svd_head_update_args {
     int step;                /* 1, 2, ...                                                */
     float lr, beta1, beta2, eps, weight_decay;
     float* loss;             /* [1] out: l before the step                               */
-    float* bhat;             /* [B] out: the forward's bhat before the step              */
+    float* bhat;             /* [B] out: the forward's bhat before the step (an input when
+                              * preact is given)                                         */
+    /* [B,M] fp32 or NULL: pre-activations W1 h + b1 of a forward already run on these hidden
+     * states with the current served weights (svd_verify_distill_args.head_preact, with that
+     * call's bhat passed in `bhat`).  Then the update skips its own forward: one kernel instead
+     * of two.  The caller guarantees that no step has changed the weights since that forward. */
+    const float* preact;
 } svd_head_update_args;
 
 /* Workspace: svd_workspace_bytes(B, 1, 1, M) bytes. */

@@ -51,7 +51,7 @@ class VerifyDistillArgs(ctypes.Structure):
         ("lambda_", _F), ("clip_c", _F), ("grad_scale", _F), ("dlogits_fp32", _I),
         ("bhat", _P), ("bk", _P), ("accept_len", _P), ("emitted", _P), ("n_emitted", _P),
         ("loss_rows", _P), ("loss_total", _P), ("dlogits", _P), ("row_info", _P),
-        ("full_k", _I), ("label_proxy", _P), ("label_full", _P),
+        ("full_k", _I), ("label_proxy", _P), ("label_full", _P), ("head_preact", _P),
     ]
 
 
@@ -63,7 +63,7 @@ class HeadUpdateArgs(ctypes.Structure):
         ("mW1", _P), ("vW1", _P), ("mb1", _P), ("vb1", _P), ("mw2", _P), ("vw2", _P),
         ("mb2", _P), ("vb2", _P), ("step", _I),
         ("lr", _F), ("beta1", _F), ("beta2", _F), ("eps", _F), ("weight_decay", _F),
-        ("loss", _P), ("bhat", _P),
+        ("loss", _P), ("bhat", _P), ("preact", _P),
     ]
 
 
@@ -263,7 +263,7 @@ class VerifyDistill:
     def __init__(self, D, T, *, head=None, bk_in=None, draft_tok=None, mode=GREEDY,
                  temperature=1.0, seed=0, step=0, lam=0.5, clip_c=1.0, grad_scale=1.0,
                  gamma=1.0, rnd=BK_CEIL, dlogits_fp32=False, row_info=False, ws=None,
-                 full_k=False, labels=False):
+                 full_k=False, labels=False, head_preact=False):
         B, k, V = D.shape
         kt = T.shape[1]
         dev = D.device
@@ -283,6 +283,9 @@ class VerifyDistill:
         # length-head labels: a / b_k as truncated verification sees it, and a / k (full-k mode)
         self.label_proxy = torch.empty(B, dtype=torch.float32, device=dev) if labels else None
         self.label_full = torch.empty(B, dtype=torch.float32, device=dev) if labels else None
+        # the head's pre-activations, for an online update that reuses this forward
+        self.head_preact = (torch.empty((B, M), dtype=torch.float32, device=dev)
+                            if head_preact and head is not None else None)
         a = VerifyDistillArgs()
         if head is not None:
             h, W1, b1, w2, b2 = head
@@ -304,6 +307,7 @@ class VerifyDistill:
         a.row_info = _ptr(self.row_info)
         a.full_k = int(bool(full_k))
         a.label_proxy, a.label_full = _ptr(self.label_proxy), _ptr(self.label_full)
+        a.head_preact = _ptr(self.head_preact)
         self.args = a
 
     def set_step(self, step: int):
@@ -323,6 +327,8 @@ class VerifyDistill:
         if self.label_proxy is not None:
             out["label_proxy"] = self.label_proxy
             out["label_full"] = self.label_full
+        if self.head_preact is not None:
+            out["head_preact"] = self.head_preact
         return out
 
 
@@ -362,12 +368,26 @@ class LengthHeadTrainer:
         """The (h, W1, b1, w2, b2) tuple for :class:`VerifyDistill` (b2 read back from device)."""
         return (h, self.W1, self.b1, self.w2, float(self.b2.item()))
 
-    def step(self, h, label, stream=None):
-        """One AdamW step on l = mean_b (bhat_b - label_b)^2; returns (loss, bhat) tensors."""
+    def step(self, h, label, stream=None, preact=None, bhat=None):
+        """One AdamW step on l = mean_b (bhat_b - label_b)^2; returns (loss, bhat) tensors.
+
+        With ``preact`` and ``bhat`` (the ``head_preact`` and ``bhat`` of a
+        :class:`VerifyDistill` step on the same h with this trainer's current weights), the
+        step reuses that forward instead of running its own."""
         if h.shape != (self.B, self.H):
             raise ValueError("h must be [B, H] = [%d, %d]" % (self.B, self.H))
+        if (preact is None) != (bhat is None):
+            raise ValueError("preact and bhat go together")
         self.step_count += 1
         a = HeadUpdateArgs()
+        bhat_buf = self.bhat
+        if preact is not None:
+            if preact.shape != (self.B, self.M) or preact.dtype != torch.float32:
+                raise ValueError("preact must be fp32 [B, M]")
+            if bhat.shape != (self.B,) or bhat.dtype != torch.float32 or not bhat.is_contiguous():
+                raise ValueError("bhat must be a contiguous fp32 [B] tensor")
+            bhat_buf = bhat            # read by the update, not written
+            a.preact = _ptr(preact.contiguous())
         lab = label.float().contiguous()
         self._label = lab   # alive until the launch is enqueued
         a.h, a.label = _ptr(_bits(h)), _ptr(lab)
@@ -377,10 +397,10 @@ class LengthHeadTrainer:
         (a.mW1, a.vW1, a.mb1, a.vb1, a.mw2, a.vw2, a.mb2, a.vb2) = [_ptr(t) for t in self.moments]
         a.step = self.step_count
         a.lr, a.beta1, a.beta2, a.eps, a.weight_decay = self.hyper
-        a.loss, a.bhat = _ptr(self.loss), _ptr(self.bhat)
+        a.loss, a.bhat = _ptr(self.loss), _ptr(bhat_buf)
         _check(lib().svd_length_head_update(ctypes.byref(a), self.ws.ptr, self.ws.nbytes,
                                             _stream(stream)), "svd_length_head_update")
-        return self.loss, self.bhat
+        return self.loss, bhat_buf
 
 
 REPORT_FIELDS = ("tau_measured", "acc", "tau_model", "eta_model", "eta_measured", "mean_bk",

@@ -58,7 +58,7 @@ __device__ __forceinline__ float delta_of(const HeadUpdateParams& p, int b) {
 // e_bm = delta_b w2_m [u_bm > 0] for its units in shared memory (from the forward's stored
 // pre-activations u, so no separate pass writes e), stages the matching h columns, and its
 // eight warps add E^T h into four 16 x 8 tiles each on the tensor cores.  The AdamW step on its
-// block of W1 follows (8-byte loads and stores).  The CTAs of column 0 also sum the w2 and b1
+// block of W1 follows, row by row (16-byte loads and stores).  The CTAs of column 0 also sum the w2 and b1
 // gradients of their units over the sequences (four threads per unit, combined in order) into
 // the workspace; the last CTA to finish (atomic ticket) applies AdamW to w2, b1 and b2 and forms
 // the loss -- only then, because every CTA reads the forward's w2 to form e.
@@ -97,6 +97,21 @@ __global__ void __launch_bounds__(256) head_back_kernel(const HeadUpdateParams p
     const bool ulive = m0 + ec < p.M;
     const float w2f = ulive ? bf16_to_f32(__ldg(p.w2 + m0 + ec)) : 0.f;   // the forward's weight
     const bool hvec = (p.H % 8 == 0) && ((reinterpret_cast<uintptr_t>(p.h) & 15) == 0) && (j0 + kTile <= p.H);
+    // The epilogue's master weights and moments (3 x 64 rows x 256 bytes) and the second
+    // chunk's operands go to L2 now, so that their loads later find them there instead of in HBM.
+    for (int x = t; x < 3 * kTile * 2; x += 256) {
+        const int arr = x / (kTile * 2), r = (x / 2) % kTile, half = x & 1;
+        const int m = m0 + r;
+        if (m < p.M && j0 + 32 * half < p.H) {
+            const float* base = arr == 0 ? p.W1m : (arr == 1 ? p.mW1 : p.vW1);
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(base + static_cast<size_t>(m) * p.H + j0 + 32 * half));
+        }
+    }
+    for (int b = kBC + t; b < p.B; b += 256) {
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.h + static_cast<size_t>(b) * p.H + j0));
+        for (int c = 0; c < kTile && m0 + c < p.M; c += 32)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.u + static_cast<size_t>(b) * p.M + m0 + c));
+    }
     float gw = 0.f, gb = 0.f;
     float acc[4][4];   // [tile nt][(g, 2tq), (g, 2tq + 1), (g + 8, 2tq), (g + 8, 2tq + 1)]
 #pragma unroll
@@ -188,35 +203,51 @@ __global__ void __launch_bounds__(256) head_back_kernel(const HeadUpdateParams p
         }
         __syncthreads();
     }
-    // AdamW epilogue on this lane's entries of W1: (m, j .. j + 1) for the rows g and g + 8 of
-    // each of its four tiles; masters and moments with 8-byte loads and stores
-    const bool wvec = (p.H % 2 == 0) &&
-                      (((reinterpret_cast<uintptr_t>(p.W1m) | reinterpret_cast<uintptr_t>(p.mW1) |
-                         reinterpret_cast<uintptr_t>(p.vW1)) & 7) == 0) &&
-                      ((reinterpret_cast<uintptr_t>(p.W1) & 3) == 0);
+    // The gradient tile goes through shared memory (the e tile's buffer) so that the AdamW
+    // epilogue walks whole rows of W1: each half-warp takes one row's 64 columns as 16-byte
+    // vectors, 256 contiguous bytes of every master and moment array per row.
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-            const int m = m0 + mb + g + 8 * half;
-            const int j = j0 + jb + nt * 8 + 2 * tq;
-            if (m >= p.M || j >= p.H) continue;
-            const size_t o = static_cast<size_t>(m) * p.H + j;
-            const float g0 = acc[nt][2 * half], g1 = acc[nt][2 * half + 1];
-            if (wvec && j + 1 < p.H) {
-                const float2 wm = *reinterpret_cast<const float2*>(p.W1m + o);
-                float2 mm = *reinterpret_cast<const float2*>(p.mW1 + o);
-                float2 vv = *reinterpret_cast<const float2*>(p.vW1 + o);
-                const float w0 = adamw(wm.x, g0, mm.x, vv.x, p);
-                const float w1 = adamw(wm.y, g1, mm.y, vv.y, p);
-                *reinterpret_cast<float2*>(p.W1m + o) = make_float2(w0, w1);
-                *reinterpret_cast<float2*>(p.mW1 + o) = mm;
-                *reinterpret_cast<float2*>(p.vW1 + o) = vv;
-                *reinterpret_cast<uint32_t*>(p.W1 + o) =
-                    f32_to_bf16_rne(w0) | (static_cast<uint32_t>(f32_to_bf16_rne(w1)) << 16);
+            const int r = mb + g + 8 * half, c = jb + nt * 8 + 2 * tq;
+            se[r][c] = acc[nt][2 * half];
+            se[r][c + 1] = acc[nt][2 * half + 1];
+        }
+    }
+    __syncthreads();
+    const bool wvec = (p.H % 4 == 0) && (j0 + kTile <= p.H) &&
+                      (((reinterpret_cast<uintptr_t>(p.W1m) | reinterpret_cast<uintptr_t>(p.mW1) |
+                         reinterpret_cast<uintptr_t>(p.vW1)) & 15) == 0) &&
+                      ((reinterpret_cast<uintptr_t>(p.W1) & 7) == 0);
+    {
+        const int c = (t & 15) * 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = (t >> 4) + 16 * q;
+            const int m = m0 + r;
+            if (m >= p.M) continue;
+            const size_t o = static_cast<size_t>(m) * p.H + j0 + c;
+            const float4 gv = *reinterpret_cast<const float4*>(&se[r][c]);
+            if (wvec) {
+                const float4 wm = *reinterpret_cast<const float4*>(p.W1m + o);
+                float4 mm = *reinterpret_cast<const float4*>(p.mW1 + o);
+                float4 vv = *reinterpret_cast<const float4*>(p.vW1 + o);
+                float4 w;
+                w.x = adamw(wm.x, gv.x, mm.x, vv.x, p);
+                w.y = adamw(wm.y, gv.y, mm.y, vv.y, p);
+                w.z = adamw(wm.z, gv.z, mm.z, vv.z, p);
+                w.w = adamw(wm.w, gv.w, mm.w, vv.w, p);
+                *reinterpret_cast<float4*>(p.W1m + o) = w;
+                *reinterpret_cast<float4*>(p.mW1 + o) = mm;
+                *reinterpret_cast<float4*>(p.vW1 + o) = vv;
+                *reinterpret_cast<uint2*>(p.W1 + o) =
+                    make_uint2(f32_to_bf16_rne(w.x) | (static_cast<uint32_t>(f32_to_bf16_rne(w.y)) << 16),
+                               f32_to_bf16_rne(w.z) | (static_cast<uint32_t>(f32_to_bf16_rne(w.w)) << 16));
             } else {
-                const float gg[2] = {g0, g1};
-                for (int jj = 0; jj < 2 && j + jj < p.H; ++jj) {
+                const float gg[4] = {gv.x, gv.y, gv.z, gv.w};
+                for (int jj = 0; jj < 4; ++jj) {
+                    if (j0 + c + jj >= p.H) break;
                     float mm = p.mW1[o + jj], vv = p.vW1[o + jj];
                     const float w = adamw(p.W1m[o + jj], gg[jj], mm, vv, p);
                     p.W1m[o + jj] = w;

@@ -7,12 +7,17 @@
 // gamma = 1.0; Referee Report minor comment 2: b_k = clamp(floor(bhat * k), 1, k)).
 //
 // The projection h [B,H] x W1^T [H,M] is a small dense contraction (2*B*H*M flops, 0.27 GFLOP
-// at B=128, H=4096, M=256) on the tensor cores: bf16 operands, fp32 accumulation.  The grid is
-// (16-sequence tiles) x (64-unit tiles) x (K splits); each CTA stages its operand slices in
-// shared memory with 16-byte loads and its 8 warps each accumulate one 16x8 output tile.  Split
-// partials land in the workspace; the last CTA of an output tile (atomic ticket, no waiting) adds
-// them in split order, applies bias, ReLU and w2, and the last tile adds the per-tile logits in
-// tile order and applies the sigmoid and the b_k map.  Every sum has a fixed order.
+// at B=128, H=4096, M=256) on the tensor cores: bf16 operands, fp32 accumulation.  Two forms:
+//   * units (H a multiple of 16, 16-byte aligned h and W1): the work units of svd_head_unit.cuh,
+//     one CTA each -- the same units the fused verify-and-distill call runs inside its row pass,
+//     so both give the same bhat and b_k;
+//   * split (any shape): grid (16-sequence tiles) x (64-unit tiles) x (K splits); each CTA stages
+//     its operand slices in shared memory with element-wise 16-byte loads and its 8 warps each
+//     accumulate one 16x8 output tile.  Split partials land in the workspace; the last CTA of an
+//     output tile (atomic ticket, no waiting) adds them in split order, applies bias, ReLU and
+//     w2, and the last tile adds the per-tile logits in tile order and applies the sigmoid and
+//     the b_k map.
+// Every sum has a fixed order in both.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -173,152 +178,9 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_kernel(const HeadPara
     if (t == 0) p.hdr->head_ticket = 0u;
 }
 
-// ------------------------------------------------------------------------------------------
-// Cluster form for H a multiple of 16 and 16-byte aligned h, W1: the K splits of a 16 x 64 output
-// tile are the 8 CTAs of a cluster.  Each stages its h and W1 slices with one bulk copy per row
-// (no multicast) on one mbarrier, runs the same tensor-core tiles, and sends its partial tile to
-// rank 0's shared memory; rank 0 adds the partials in rank order, applies bias, ReLU and w2, and
-// writes the tile's per-sequence logits.  The last of the M/64 tiles of a 16-sequence block (a
-// ticket per block) adds them in tile order and applies the sigmoid and the b_k map.  One
-// global round trip and one ticket instead of split partials through global memory.
-// ------------------------------------------------------------------------------------------
 namespace {
-
-constexpr int kHeadCl = 8;             // CTAs per cluster = K splits
-constexpr int kKC2 = 512;              // K columns staged per round
-constexpr int kLd2 = kKC2 + kPad;      // 1040-byte rows: 16-byte aligned, conflict-free
-constexpr size_t kHeadClSmem = static_cast<size_t>(kHeadTileB + kHeadTileM) * kLd2 * 2 + 16;
-static_assert(static_cast<size_t>(kHeadCl) * kHeadTileB * kHeadTileM * 4 <=
-              static_cast<size_t>(kHeadTileB + kHeadTileM) * kLd2 * 2,
-              "the partial tiles of the cluster fit in rank 0's staging area");
-constexpr uint64_t kHeadWaitNs = 1000000000ull;   // 1 s bound on the staging wait
-
+constexpr uint64_t kHeadWaitNs = 1000000000ull;   // 1 s bound on a unit's staging wait
 }  // namespace
-
-__global__ void __launch_bounds__(kWarps * 32) length_head_cluster_kernel(const HeadParams p) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    uint16_t* hs = reinterpret_cast<uint16_t*>(smem_raw);
-    uint16_t* ws = hs + kHeadTileB * kLd2;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(ws + kHeadTileM * kLd2);
-    float* red = reinterpret_cast<float*>(smem_raw);   // rank 0, after the staging is consumed
-    __shared__ float pre[kHeadTileB][kHeadTileM + 1];
-    __shared__ int flag;
-
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const uint32_t rank = cluster_rank();
-    const int bt = blockIdx.y, mt = blockIdx.z;
-    const int b0 = bt * kHeadTileB, m0 = mt * kHeadTileM;
-    const int g = lane >> 2, tq = lane & 3;
-    const int k_lo = min(p.H, static_cast<int>(rank) * p.ks), k_hi = min(p.H, k_lo + p.ks);
-    if (t == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t phase = 0;
-    bool dead = false;
-    for (int c0 = k_lo; c0 < k_hi; c0 += kKC2) {
-        const int len = min(k_hi, c0 + kKC2) - c0;   // a multiple of 16
-        // rows past the batch or the units read as zeros
-        for (int x = t; x < (kHeadTileB + kHeadTileM) * (len / 8); x += blockDim.x) {
-            const int r = x / (len / 8), cv = (x % (len / 8)) * 8;
-            const bool valid = r < kHeadTileB ? (b0 + r < p.B) : (m0 + r - kHeadTileB < p.M);
-            if (!valid) *reinterpret_cast<uint4*>(hs + r * kLd2 + cv) = make_uint4(0, 0, 0, 0);
-        }
-        if (t == 0) {
-            const int nh = max(0, min(kHeadTileB, p.B - b0)), nw = max(0, min(kHeadTileM, p.M - m0));
-            mbar_arrive_expect_tx(bar, static_cast<uint32_t>((nh + nw) * len * 2));
-        }
-        __syncthreads();
-        if (t < kHeadTileB + kHeadTileM) {
-            const uint32_t bytes = static_cast<uint32_t>(len) * 2u;
-            if (t < kHeadTileB) {
-                if (b0 + t < p.B)
-                    bulk_load(hs + t * kLd2, p.h + static_cast<size_t>(b0 + t) * p.H + c0, bytes, bar);
-            } else {
-                const int r = t - kHeadTileB;
-                if (m0 + r < p.M)
-                    bulk_load(ws + r * kLd2, p.W1 + static_cast<size_t>(m0 + r) * p.H + c0, bytes, bar);
-            }
-        }
-        if (!dead && !mbar_wait_bounded(bar, phase, kHeadWaitNs)) {
-            dead = true;
-            set_device_error(&p.hdr->status, SVD_ERR_TIMEOUT);
-        }
-        phase ^= 1u;
-        const uint16_t* wrow = ws + (warp * 8 + g) * kLd2;
-        for (int kk = 0; kk < len; kk += 16) {
-            uint32_t a[4], bf[2];
-            a[0] = *reinterpret_cast<const uint32_t*>(hs + g * kLd2 + kk + 2 * tq);
-            a[1] = *reinterpret_cast<const uint32_t*>(hs + (g + 8) * kLd2 + kk + 2 * tq);
-            a[2] = *reinterpret_cast<const uint32_t*>(hs + g * kLd2 + kk + 2 * tq + 8);
-            a[3] = *reinterpret_cast<const uint32_t*>(hs + (g + 8) * kLd2 + kk + 2 * tq + 8);
-            bf[0] = *reinterpret_cast<const uint32_t*>(wrow + kk + 2 * tq);
-            bf[1] = *reinterpret_cast<const uint32_t*>(wrow + kk + 2 * tq + 8);
-            mma_bf16_16816(acc, a, bf);
-        }
-        __syncthreads();
-    }
-    // every rank is done with its staging: the partial tiles go to rank 0
-    cluster_sync();
-    {
-        const int col = warp * 8 + 2 * tq;
-        const int rows[2] = {g, g + 8};
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const size_t o = (static_cast<size_t>(rank) * kHeadTileB + rows[h2]) * kHeadTileM + col;
-            dsmem_st_f32(dsmem_map(red + o, 0), acc[2 * h2]);
-            dsmem_st_f32(dsmem_map(red + o + 1, 0), acc[2 * h2 + 1]);
-        }
-    }
-    cluster_sync();
-    if (rank != 0) return;
-    for (int o = t; o < kHeadTileB * kHeadTileM; o += blockDim.x) {
-        const int r = o / kHeadTileM, col = o % kHeadTileM;
-        const int b = b0 + r, m = m0 + col;
-        float a = 0.f;
-        if (b < p.B && m < p.M) {
-            for (int q = 0; q < kHeadCl; ++q) a += red[(q * kHeadTileB + r) * kHeadTileM + col];
-            if (p.b1) a += __ldg(p.b1 + m);
-            if (p.u_out) p.u_out[static_cast<size_t>(b) * p.M + m] = a;
-            const float w2 = __uint_as_float(static_cast<uint32_t>(__ldg(p.w2 + m)) << 16);
-            a = w2 * fmaxf(a, 0.f);
-        }
-        pre[r][col] = a;
-    }
-    __syncthreads();
-    for (int r = warp * 2; r < warp * 2 + 2; ++r) {
-        float z = pre[r][lane] + pre[r][lane + 32];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-        if (lane == 0 && b0 + r < p.B) p.zpart[static_cast<size_t>(mt) * p.B + b0 + r] = z;
-    }
-    // the last of this block's unit tiles finishes its 16 sequences; the lanes that wrote
-    // partial logits fence them before the ticket, the lanes that read them after it
-    if (lane == 0) __threadfence();
-    __syncthreads();
-    if (t == 0) {
-        const uint32_t old = atomicAdd(&p.tile_ticket[bt], 1u);
-        flag = (old + 1u == gridDim.z) ? 1 : 0;
-    }
-    __syncthreads();
-    if (!flag) return;
-    if (t < kHeadTileB) __threadfence();
-    if (t < kHeadTileB && b0 + t < p.B) {
-        const int b = b0 + t;
-        float z = p.b2_dev ? *p.b2_dev : p.b2;
-        for (int q = 0; q < static_cast<int>(gridDim.z); ++q) z += __ldcg(p.zpart + static_cast<size_t>(q) * p.B + b);
-        const float bhat = 1.f / (1.f + expf(-z));
-        const float target = p.gamma * bhat * static_cast<float>(p.k);
-        const float rr = p.rnd == 0 ? ceilf(target) : floorf(target);
-        int bk = static_cast<int>(fminf(fmaxf(rr, 1.f), static_cast<float>(p.k)));
-        if (!(rr == rr)) bk = 1;  // non-finite hidden states
-        if (p.bhat) p.bhat[b] = bhat;
-        if (p.bk) p.bk[b] = bk;
-    }
-    if (t == 0) p.tile_ticket[bt] = 0u;
-}
 
 // The head as independent work units (svd_head_unit.cuh), one CTA per unit: the same units the
 // fused verify-and-distill pass runs inside its row pass, so both give the same bhat and b_k.
@@ -345,9 +207,11 @@ size_t head_unit_stage_bytes(int ks) {
 
 int launch_length_head(const HeadParams& p, void* stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool cluster_form = (p.H % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.h) & 15) == 0) &&
-                              ((reinterpret_cast<uintptr_t>(p.W1) & 15) == 0);
-    if (!cluster_form) {
+    // units need H a multiple of 16 and 16-byte aligned rows (bulk copies); otherwise the
+    // split form with element-wise staging
+    const bool units_form = (p.H % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.h) & 15) == 0) &&
+                            ((reinterpret_cast<uintptr_t>(p.W1) & 15) == 0);
+    if (!units_form) {
         dim3 grid((p.B + kHeadTileB - 1) / kHeadTileB, (p.M + kHeadTileM - 1) / kHeadTileM, p.nsplit);
         length_head_kernel<<<grid, kWarps * 32, 0, st>>>(p);
         return static_cast<int>(cudaGetLastError());

@@ -234,13 +234,14 @@ svd_status svd_verify_distill(const svd_verify_distill_args* a, void* ws, size_t
     const bool fuse_head = head && a->B <= kRowCompactMaxB && a->H % 16 == 0 && aligned16(a->h) &&
                            aligned16(a->W1);
     HeadParams hp;
-    if (fuse_head) {
+    if (head) {
         hp = head_params(a->h, a->W1, a->b1, a->w2, a->b2, a->B, a->H, a->M, a->k, a->gamma,
                          a->rnd, a->bhat, a->bk, w);
-    } else if (head) {
-        s = run_head(a->h, a->W1, a->b1, a->w2, a->b2, a->B, a->H, a->M, a->k, a->gamma, a->rnd,
-                     a->bhat, a->bk, w, stream);
-        if (s != SVD_OK) return s;
+        hp.u_out = a->head_preact;
+        if (!fuse_head) {
+            s = from_cuda(launch_length_head(hp, stream));
+            if (s != SVD_OK) return s;
+        }
     } else if (a->bk != a->bk_in) {
         if (cudaMemcpyAsync(a->bk, a->bk_in, sizeof(int32_t) * a->B, cudaMemcpyDeviceToDevice,
                             static_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -273,7 +274,10 @@ svd_status svd_length_head_update(const svd_head_update_args* a, void* ws, size_
     char* base = static_cast<char*>(ws);
     float* u = reinterpret_cast<float*>(base + L.u);
     float* e = reinterpret_cast<float*>(base + L.e);
-    // forward on the served weights, keeping the pre-activations
+    // forward on the served weights, keeping the pre-activations -- unless the caller passes
+    // those of a forward already run (then bhat is that forward's, an input)
+    const bool have_fwd = a->preact != nullptr;
+    if (have_fwd) u = const_cast<float*>(a->preact);
     HeadParams hp;
     hp.h = a->h; hp.W1 = a->W1; hp.b1 = a->b1; hp.w2 = a->w2; hp.b2 = 0.f;
     hp.B = a->B; hp.H = a->H; hp.M = a->M; hp.k = 1;
@@ -283,8 +287,10 @@ svd_status svd_length_head_update(const svd_head_update_args* a, void* ws, size_
     hp.nsplit = head_nsplit(a->B, a->M);
     const int per = (a->H + hp.nsplit - 1) / hp.nsplit;
     hp.ks = (per + 15) & ~15;
-    s = from_cuda(launch_length_head(hp, stream));
-    if (s != SVD_OK) return s;
+    if (!have_fwd) {
+        s = from_cuda(launch_length_head(hp, stream));
+        if (s != SVD_OK) return s;
+    }
     HeadUpdateParams p;
     p.h = a->h; p.label = a->label; p.bhat = a->bhat; p.u = u; p.e = e;
     p.ticket = &w.hdr->update_ticket;

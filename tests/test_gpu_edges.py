@@ -270,3 +270,33 @@ def test_empty_batch():
     bk = torch.empty((0,), dtype=torch.int32, device="cuda")
     assert api.lib().svd_verify(None, None, None, None, 0, 4, 4, 64, 0, 1.0, 0, 0, None, None,
                                 None, None, None, 0, None) == 0
+
+
+@pytest.mark.parametrize("B,H,M,V", [(5, 272, 100, 20000), (17, 4096, 64, 16392),
+                                     (40, 1000, 300, 40960), (3, 16, 1, 151936)])
+def test_fused_head_ragged_shapes(B, H, M, V):
+    """The length head inside the row pass on partial sequence / unit tiles (B % 16, M % 64 not
+    zero), and the separate head kernel before it where H % 16 != 0: b_k, bhat and everything
+    downstream against the oracle."""
+    k = 6
+    g = torch.Generator().manual_seed(B * 7 + H + M)
+    h = (3 * torch.randn((B, H), generator=g)).to(torch.bfloat16)
+    W1 = (0.05 * torch.randn((M, H), generator=g)).to(torch.bfloat16)
+    w2 = (0.1 * torch.randn((M,), generator=g)).to(torch.bfloat16)
+    b1 = 0.01 * torch.randn((M,), generator=g)
+    D, T = make_case(B, k, k, V, seed=B + M, sigma=0.9)
+    vd = api.VerifyDistill(cuda(D), cuda(T), head=(cuda(h), cuda(W1), cuda(b1), cuda(w2), 0.05),
+                           lam=0.5, clip_c=0.5, row_info=True, head_preact=True)
+    vd()
+    torch.cuda.synchronize()
+    assert api.svd_get_device_error(vd.ws) == 0
+    out = vd.outputs()
+    rb, rk, _ = oracle.length_head(h, W1, b1.double().numpy(), w2, 0.05, k, 1.0, 0)
+    near = P.bk_near_integer(rb, k)
+    bk = out["bk"].cpu().numpy()
+    assert np.array_equal(bk[~near], rk[~near])
+    P.assert_close(out["bhat"].cpu().numpy(), rb, "bhat", rtol=1e-4, atol=1e-6)
+    # the pre-activations W1 h + b1 the head hands to an online update
+    pre = (h.double() @ W1.double().T + b1.double()).numpy()
+    P.assert_close(out["head_preact"].cpu().numpy(), pre, "head_preact", rtol=1e-4, atol=1e-4)
+    full_compare(vd, D, T, bk, lam=0.5, clip_c=0.5)

@@ -96,3 +96,36 @@ def test_bad_arguments():
     import ctypes
     assert L.svd_length_head_update(None, None, 0, None) == 1
     assert L.svd_length_head_update(ctypes.byref(a), None, 0, None) == 1   # B = 0, null pointers
+
+
+def test_update_reusing_the_verification_forward():
+    """The fused call's head pre-activations and bhat stand in for the update's own forward:
+    the step then matches the oracle's (which recomputes the forward) as closely as a step
+    with its own forward does."""
+    w = syn.WORKLOADS["greedy_qwen_b32"]
+    D, T = syn.make_logits(w)
+    h, W1, b1, w2, b2 = syn.make_head(w)
+    tr = api.LengthHeadTrainer(W1.cuda(), b1.cuda(), w2.cuda(), b2, w.B, lr=LR)
+    hd = h.cuda()
+    for step in (1, 2):
+        vd = api.VerifyDistill(D.cuda(), T.cuda(), head=tr.head(hd), lam=w.lam, clip_c=w.clip_c,
+                               labels=True, head_preact=True)
+        vd()
+        torch.cuda.synchronize()
+        label = vd.label_proxy.clone()
+        st = _oracle_state(tr)
+        ref = oracle.length_head_update(h, label.cpu().double().numpy(), tr.W1.cpu(),
+                                        st["b1m"].copy(), tr.w2.cpu(), float(st["b2m"][0]), st,
+                                        tr.step_count + 1, lr=LR)
+        loss, bhat = tr.step(hd, label, preact=vd.head_preact, bhat=vd.bhat)
+        torch.cuda.synchronize()
+        assert loss.item() == pytest.approx(ref["loss"], rel=2e-5)
+        np.testing.assert_allclose(bhat.cpu().numpy(), ref["bhat"], rtol=2e-5, atol=1e-6)
+        for name, gpu, gname in (("W1m", tr.W1m, "gW1"), ("b1m", tr.b1, "gb1"), ("w2m", tr.w2m, "gw2")):
+            got, want = _np(gpu), st[name]
+            g = np.abs(ref[gname])
+            ambiguous = g < 1e-4 * g.max()
+            bad = (np.abs(got - want) > 1e-3 * LR + 1e-6 * np.abs(want)) & ~ambiguous
+            assert not bad.any(), (name, step, int(bad.sum()))
+        np.testing.assert_allclose(_np(tr.moments[0]), st["mW1"], rtol=1e-3, atol=1e-9)
+        assert torch.equal(tr.W1, tr.W1m.to(torch.bfloat16))
