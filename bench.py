@@ -51,7 +51,8 @@ METRIC = "verified draft tokens/s and fused-pass HBM GB/s (% of B200 peak) at B=
 UNIT = "verified draft tokens/s"
 CSRC = os.path.join(ROOT, "speculative_decoding_verify_distill_b200", "csrc")
 # the sources the row-pass kernel is compiled from (its recorded DRAM traffic is tied to them)
-KERNEL_SRCS = [os.path.join(CSRC, f) for f in ("verify_distill.cu", "svd_device.cuh", "svd_internal.h")]
+KERNEL_SRCS = [os.path.join(CSRC, f) for f in ("verify_distill.cu", "svd_device.cuh", "svd_internal.h",
+                                                "svd_head_unit.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "row_pass_kernel_ragged_qwen_b128.md")
 
 

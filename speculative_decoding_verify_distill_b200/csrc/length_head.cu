@@ -20,7 +20,10 @@
 // Every sum has a fixed order in both.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
+#include <mutex>
+#include <vector>
 
 #include "svd_device.cuh"
 #include "svd_head_unit.cuh"
@@ -190,6 +193,10 @@ __global__ void __launch_bounds__(kWarps * 32) length_head_units_kernel(const He
     extern __shared__ __align__(128) unsigned char smem_raw[];
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + stage_bytes);
     __shared__ int flag;
+    // launched as a programmatic dependent of the preceding kernel: nothing is read before it
+    // has finished; the kernel after this one may be scheduled at once (it waits likewise)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
@@ -217,16 +224,37 @@ int launch_length_head(const HeadParams& p, void* stream) {
         return static_cast<int>(cudaGetLastError());
     }
     // one chunk per unit when it fits in 100 KB, else chunks of what does
+    constexpr size_t kMaxStage = 100 * 1024;
     size_t stage = head_unit_stage_bytes(p.ks);
-    if (stage > 100 * 1024) stage = 100 * 1024;
+    if (stage > kMaxStage) stage = kMaxStage;
     stage = (stage + 127) & ~size_t(127);
     const size_t smem = stage + 16;
-    cudaError_t err = cudaFuncSetAttribute(length_head_units_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-    if (err != cudaSuccess) return static_cast<int>(err);
-    length_head_units_kernel<<<head_units(p), kWarps * 32, smem, st>>>(p, static_cast<uint32_t>(stage));
-    return static_cast<int>(cudaGetLastError());
+    {
+        // the dynamic shared-memory limit, raised to the largest stage once per device
+        static std::mutex lock;
+        static std::vector<int> done;
+        int dev = 0;
+        cudaError_t err = cudaGetDevice(&dev);
+        if (err != cudaSuccess) return static_cast<int>(err);
+        std::lock_guard<std::mutex> guard(lock);
+        if (std::find(done.begin(), done.end(), dev) == done.end()) {
+            err = cudaFuncSetAttribute(length_head_units_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kMaxStage + 16));
+            if (err != cudaSuccess) return static_cast<int>(err);
+            done.push_back(dev);
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(head_units(p)), 1, 1);
+    cfg.blockDim = dim3(kWarps * 32, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    return static_cast<int>(cudaLaunchKernelEx(&cfg, length_head_units_kernel, p, static_cast<uint32_t>(stage)));
 }
 
 // ------------------------------------------------------------------------------------------

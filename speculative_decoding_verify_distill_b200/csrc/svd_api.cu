@@ -299,8 +299,8 @@ svd_status svd_length_head_update(const svd_head_update_args* a, void* ws, size_
     p.mW1 = a->mW1; p.vW1 = a->vW1; p.mb1 = a->mb1; p.vb1 = a->vb1;
     p.mw2 = a->mw2; p.vw2 = a->vw2; p.mb2 = a->mb2; p.vb2 = a->vb2;
     p.lr = a->lr; p.beta1 = a->beta1; p.beta2 = a->beta2; p.eps = a->eps; p.wd = a->weight_decay;
-    p.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(a->beta1), a->step));
-    p.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(a->beta2), a->step));
+    p.step_size = static_cast<float>(a->lr / (1.0 - std::pow(static_cast<double>(a->beta1), a->step)));
+    p.rsqrt_bc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(a->beta2), a->step)));
     p.loss = a->loss;
     return from_cuda(launch_head_update(p, stream));
 }

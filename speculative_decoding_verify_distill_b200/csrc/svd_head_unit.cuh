@@ -52,7 +52,8 @@ __host__ __device__ inline int head_chunk_cols(size_t smem_bytes) {
 
 // One unit, executed by all threads of the calling CTA (H a multiple of 16; h and W1 16-byte
 // aligned).  The split's K range is staged in chunks: one bulk copy (1-D TMA, no multicast) per
-// row of h and of W1 into `stage` (smem_bytes of this CTA's shared memory), completing on the
+// row of h and of W1, issued by the lanes of warp 0 in turn, into `stage` (smem_bytes of this
+// CTA's shared memory), completing on the
 // mbarrier `bar` (count 1; `phase` is its parity, flipped per chunk), then the warps take the
 // eight 16 x 8 blocks of hidden units m0 + 8j .. m0 + 8j + 7 in turn and accumulate them over
 // the chunk from shared memory.  A chunk costs one round trip to memory.  `flag` is one int of
@@ -98,14 +99,19 @@ __device__ __forceinline__ bool head_unit(const HeadParams& p, int u, int* flag,
     for (int ch = 0; ch < nchunk; ++ch) {
         const int c0 = k_lo + ch * cw, c1 = min(k_hi, c0 + cw);
         __syncthreads();      // every read of the previous chunk (and the zero rows) is done
-        if (t == 0) {
+        if (warp == 0) {
+            // lane 0 announces the chunk's bytes, then the 32 lanes issue its row copies
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             const uint32_t row_bytes = static_cast<uint32_t>(c1 - c0) * 2u;
-            mbar_arrive_expect_tx(bar, row_bytes * static_cast<uint32_t>(nrow_h + nrow_w));
-            for (int r = 0; r < nrow_h; ++r)
-                bulk_load(hs + r * ld, p.h + static_cast<size_t>(b0 + r) * p.H + c0, row_bytes, bar);
-            for (int r = 0; r < nrow_w; ++r)
-                bulk_load(ws + r * ld, p.W1 + static_cast<size_t>(m0 + r) * p.H + c0, row_bytes, bar);
+            if (lane == 0) mbar_arrive_expect_tx(bar, row_bytes * static_cast<uint32_t>(nrow_h + nrow_w));
+            __syncwarp();
+            for (int r = lane; r < nrow_h + nrow_w; r += 32) {
+                if (r < nrow_h)
+                    bulk_load(hs + r * ld, p.h + static_cast<size_t>(b0 + r) * p.H + c0, row_bytes, bar);
+                else
+                    bulk_load(ws + (r - nrow_h) * ld, p.W1 + static_cast<size_t>(m0 + r - nrow_h) * p.H + c0,
+                              row_bytes, bar);
+            }
         }
         if (ok && !mbar_wait_bounded(bar, phase, wait_limit_ns)) {
             ok = false;
@@ -157,34 +163,44 @@ __device__ __forceinline__ bool head_unit(const HeadParams& p, int u, int* flag,
     __syncthreads();
     if (!*flag) return ok;
     __threadfence();
-    // one warp per row of the tile; lane: units lane and lane + 32 (fixed orders)
-    for (int r = warp; r < kHeadTileB; r += nw) {
+    // sixteen threads per row of the tile, four units each (m0 + l + 16 i): the split partials
+    // of all four in flight eight splits at a time, added in split order; then b1, ReLU and w2,
+    // and the row's sixteen threads combined by a fixed butterfly
+    for (int o = t; o < kHeadTileB * 16; o += blockDim.x) {
+        const int r = o >> 4, l = o & 15;
         const int b = b0 + r;
-        float zz = 0.f;
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
         if (b < p.B) {
+            for (int z0 = 0; z0 < p.nsplit; z0 += 8) {
+                float v[8][4];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int m = m0 + lane + 32 * half;
-                float a = 0.f;
-                if (m < p.M) {
-                    // all split partials in flight at once (at most 16), then added in split order
-                    float v[16];
+                for (int z = 0; z < 8; ++z) {
+                    const float* src = p.part + (static_cast<size_t>(z0 + z) * p.B + b) * p.M + m0 + l;
 #pragma unroll
-                    for (int z = 0; z < 16; ++z)
-                        v[z] = z < p.nsplit ? __ldcg(p.part + (static_cast<size_t>(z) * p.B + b) * p.M + m) : 0.f;
-#pragma unroll
-                    for (int z = 0; z < 16; ++z) a += v[z];
-                    if (p.b1) a += __ldg(p.b1 + m);
-                    if (p.u_out) p.u_out[static_cast<size_t>(b) * p.M + m] = a;
-                    const float w2 = __uint_as_float(static_cast<uint32_t>(__ldg(p.w2 + m)) << 16);
-                    a = w2 * fmaxf(a, 0.f);
+                    for (int i = 0; i < 4; ++i)
+                        v[z][i] = (z0 + z < p.nsplit && m0 + l + 16 * i < p.M) ? __ldcg(src + 16 * i) : 0.f;
                 }
-                zz += a;
+#pragma unroll
+                for (int z = 0; z < 8; ++z)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) a[i] += v[z][i];
+            }
+        }
+        float zz = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int m = m0 + l + 16 * i;
+            if (b < p.B && m < p.M) {
+                float x = a[i];
+                if (p.b1) x += __ldg(p.b1 + m);
+                if (p.u_out) p.u_out[static_cast<size_t>(b) * p.M + m] = x;
+                const float w2 = __uint_as_float(static_cast<uint32_t>(__ldg(p.w2 + m)) << 16);
+                zz += w2 * fmaxf(x, 0.f);
             }
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
-        if (lane == 0 && b < p.B) p.zpart[static_cast<size_t>(mt) * p.B + b] = zz;
+        for (int o2 = 8; o2 > 0; o2 >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o2);
+        if (l == 0 && b < p.B) p.zpart[static_cast<size_t>(mt) * p.B + b] = zz;
     }
     if (t == 0) p.tile_ticket[bt * MT + mt] = 0u;
     // ------------------------------------------------ last tile of the sequence tile

@@ -151,13 +151,14 @@ struct HeadUpdateParams {
     const float* label;
     const float* bhat;
     const float* u;          // [B, M] pre-activations of the forward
-    float* e;                // workspace: [2, M] w2 and b1 gradients
+    float* e;                // workspace: [M] the new w2 masters, until the last CTA copies them
     uint32_t* ticket;        // backward CTAs finished (back to zero after the step)
     int B, H, M;
     float *W1m, *b1, *w2m, *b2;
     uint16_t *W1, *w2;
     float *mW1, *vW1, *mb1, *vb1, *mw2, *vw2, *mb2, *vb2;
-    float lr, beta1, beta2, eps, wd, bc1, bc2;   // bc = 1 - beta^step
+    float lr, beta1, beta2, eps, wd;
+    float step_size, rsqrt_bc2;   // lr / (1 - beta1^step), 1 / sqrt(1 - beta2^step)
     float* loss;
 };
 int launch_head_update(const HeadUpdateParams& p, void* stream);

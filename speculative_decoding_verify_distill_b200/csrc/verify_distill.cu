@@ -227,6 +227,10 @@ __global__ void __launch_bounds__(NT, MINB) row_pass_kernel(const RowParams p) {
     int* spre = sbk + p.B;
     int* zpre = spre + p.B + 1;
 
+    // launched as a programmatic dependent of whatever kernel precedes it on the stream: its
+    // CTAs may be resident early, but read nothing before that grid has finished (the previous
+    // step's finalize pass resets this workspace's tickets)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // the finalize pass may be scheduled as soon as SM resources allow; it waits for this grid
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
@@ -1304,7 +1308,7 @@ int launch_row_pass(const RowParams& p, void* stream) {
                                    : pick_kernel<kXNT, kXNV, kXMB>(p.flags, aligned);
     const size_t smem = row_smem_bytes(geo, p.B);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = geo.cluster;
     attr[0].val.clusterDim.y = 1;
@@ -1322,6 +1326,11 @@ int launch_row_pass(const RowParams& p, void* stream) {
     int nclusters = cache;
     if (max_items < nclusters) nclusters = static_cast<int>(max_items > 0 ? max_items : 1);
     cfg.gridDim = dim3(geo.cluster * nclusters, 1, 1);
+    // a programmatic dependent of the preceding kernel (the kernel waits for it first thing):
+    // the launch latency overlaps that kernel's tail
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
     RowParams q = p;
     q.chunk = geo.chunk;
     err = cudaLaunchKernelEx(&cfg, fn, q);
