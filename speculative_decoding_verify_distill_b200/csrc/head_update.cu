@@ -69,8 +69,9 @@ __device__ __forceinline__ float delta_of(const HeadUpdateParams& p, int b) {
 // units over the sequences (in the same fragments; per warp the four lanes of a unit combined
 // by a fixed butterfly, then the two halves) and step the fp32 masters and moments of w2 and
 // b1 themselves (nothing else in the kernel reads them); only the bf16 w2, which every CTA
-// reads to form e, waits for the last CTA to finish (atomic ticket), which copies it in.
-// CTA (0, 0) forms the loss and steps b2 while its first copies are in flight.
+// reads to form e, waits for the last CTA to take an atomic ticket (taken after the MMA, before
+// the W1 stores), which copies it in.  CTA (0, 0) forms the loss and steps b2 while its first
+// copies are in flight.
 constexpr int kBC = 128;         // sequences per chunk (one chunk up to B = 128)
 constexpr int kHLd = kTile + 8;  // bf16 row pitch of the staged h tile (16-byte rows)
 constexpr int kELd = kTile + 4;  // fp32 row pitch of the u tile (fragment reads on distinct banks)
@@ -116,6 +117,7 @@ __global__ void __launch_bounds__(256, 2) head_back_kernel(const HeadUpdateParam
         back_smem + sizeof(float) * kBC * kELd + sizeof(uint16_t) * kBC * kHLd);
     __shared__ float sdelta[kBC];
     __shared__ float sg[2][2][kTile];                     // [half][w2 / b1] gradients of the units
+    __shared__ float sp[6][kTile];                        // column 0: w2 / b1 masters and moments
     __shared__ int last;
     // launched as a programmatic dependent of the preceding kernel: nothing is read before it
     // has finished
@@ -170,6 +172,18 @@ __global__ void __launch_bounds__(256, 2) head_back_kernel(const HeadUpdateParam
         cp_async_commit();
     };
     stage_chunk(0);
+    // delta of the first chunk's sequences while its copies fly
+    for (int r = t; r < kBC; r += 256) sdelta[r] = r < min(kBC, p.B) ? delta_of(p, r) : 0.f;
+    if (col0 && t < kTile && m0 + t < p.M) {
+        // column 0: its units' w2 and b1 masters and moments, for the AdamW steps after the MMA
+        const int m = m0 + t;
+        sp[0][t] = p.w2m[m];
+        sp[1][t] = p.mw2[m];
+        sp[2][t] = p.vw2[m];
+        sp[3][t] = p.b1[m];
+        sp[4][t] = p.mb1[m];
+        sp[5][t] = p.vb1[m];
+    }
     // the forward's w2 of this thread's two fragment units (rows g and g + 8 of its tiles)
     const float w2a = m0 + mb + g < p.M ? bf16_to_f32(__ldg(p.w2 + m0 + mb + g)) : 0.f;
     const float w2b = m0 + mb + g + 8 < p.M ? bf16_to_f32(__ldg(p.w2 + m0 + mb + g + 8)) : 0.f;
@@ -206,6 +220,7 @@ __global__ void __launch_bounds__(256, 2) head_back_kernel(const HeadUpdateParam
         const int nb = min(kBC, p.B - b0);
         if (b0 > 0) {
             stage_chunk(b0);
+            for (int r = t; r < kBC; r += 256) sdelta[r] = r < nb ? delta_of(p, b0 + r) : 0.f;
             cp_async_wait<0>();   // (the W1 block, committed earlier, has landed too)
         } else {
             cp_async_wait<0>();
@@ -222,7 +237,6 @@ __global__ void __launch_bounds__(256, 2) head_back_kernel(const HeadUpdateParam
             }
             cp_async_commit();    // in flight while the tensor cores run
         }
-        for (int r = t; r < kBC; r += 256) sdelta[r] = r < nb ? delta_of(p, b0 + r) : 0.f;
         __syncthreads();
         // dW1 tile += E^T h over the chunk's sequences, 16 at a time, on the tensor cores
         // (mma.sync m16n8k16, fp32 accumulation).  e_bm = delta_b w2_m [u_bm > 0] is formed
@@ -271,6 +285,50 @@ __global__ void __launch_bounds__(256, 2) head_back_kernel(const HeadUpdateParam
             }
         }
         __syncthreads();
+    }
+    // column 0: this tile's units' w2 / b1 gradients, summed over the sequences in a fixed
+    // order, and the AdamW steps of their fp32 masters and moments; the new w2 goes to the
+    // workspace until every CTA has read the old one
+    if (col0) {
+        // the four lanes of a unit (tq = 0..3) hold disjoint rows of the warp's half
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            gw[i] += __shfl_xor_sync(0xffffffffu, gw[i], 1);
+            gw[i] += __shfl_xor_sync(0xffffffffu, gw[i], 2);
+            gb[i] += __shfl_xor_sync(0xffffffffu, gb[i], 1);
+            gb[i] += __shfl_xor_sync(0xffffffffu, gb[i], 2);
+        }
+        if (tq == 0) {
+            sg[kh][0][mb + g] = gw[0];
+            sg[kh][0][mb + g + 8] = gw[1];
+            sg[kh][1][mb + g] = gb[0];
+            sg[kh][1][mb + g + 8] = gb[1];
+        }
+        __syncthreads();
+        if (t < kTile && m0 + t < p.M) {
+            const int m = m0 + t;
+            const float a = sg[0][0][t] + sg[1][0][t], c = sg[0][1][t] + sg[1][1][t];
+            float mm = sp[1][t], vv = sp[2][t];
+            const float w2n = adamw(sp[0][t], a, mm, vv, p);
+            float mb = sp[4][t], vb = sp[5][t];
+            const float b1n = adamw(sp[3][t], c, mb, vb, p);
+            p.w2m[m] = w2n;
+            p.mw2[m] = mm;
+            p.vw2[m] = vv;
+            p.b1[m] = b1n;
+            p.mb1[m] = mb;
+            p.vb1[m] = vb;
+            p.e[m] = w2n;                    // workspace: the new w2 master, [M]
+        }
+    }
+    // the ticket, before this CTA's W1 stores, so that the fence waits only for the column-0
+    // writes above; every CTA has read the forward's w2 by now.  The atomic is in flight while
+    // the epilogue runs, and the last CTA to take it publishes the new bf16 w2.
+    __syncthreads();
+    uint32_t ticket_old = 0u;
+    if (t == 0) {
+        __threadfence();
+        ticket_old = atomicAdd(p.ticket, 1u);
     }
     // The gradient tile goes through shared memory (the u tile's buffer) so that the AdamW
     // epilogue walks whole rows of W1: each half-warp takes one row's 64 columns as 16-byte
@@ -337,48 +395,7 @@ __global__ void __launch_bounds__(256, 2) head_back_kernel(const HeadUpdateParam
             }
         }
     }
-    // column 0: this tile's units' w2 / b1 gradients, summed over the sequences in a fixed
-    // order, and the AdamW steps of their fp32 masters and moments; the new w2 goes to the
-    // workspace until every CTA has read the old one
-    if (col0) {
-        // the four lanes of a unit (tq = 0..3) hold disjoint rows of the warp's half
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            gw[i] += __shfl_xor_sync(0xffffffffu, gw[i], 1);
-            gw[i] += __shfl_xor_sync(0xffffffffu, gw[i], 2);
-            gb[i] += __shfl_xor_sync(0xffffffffu, gb[i], 1);
-            gb[i] += __shfl_xor_sync(0xffffffffu, gb[i], 2);
-        }
-        if (tq == 0) {
-            sg[kh][0][mb + g] = gw[0];
-            sg[kh][0][mb + g + 8] = gw[1];
-            sg[kh][1][mb + g] = gb[0];
-            sg[kh][1][mb + g + 8] = gb[1];
-        }
-        __syncthreads();
-        if (t < kTile && m0 + t < p.M) {
-            const int m = m0 + t;
-            const float a = sg[0][0][t] + sg[1][0][t], c = sg[0][1][t] + sg[1][1][t];
-            float mm = p.mw2[m], vv = p.vw2[m];
-            const float w2n = adamw(p.w2m[m], a, mm, vv, p);
-            float mb = p.mb1[m], vb = p.vb1[m];
-            const float b1n = adamw(p.b1[m], c, mb, vb, p);
-            p.w2m[m] = w2n;
-            p.mw2[m] = mm;
-            p.vw2[m] = vv;
-            p.b1[m] = b1n;
-            p.mb1[m] = mb;
-            p.vb1[m] = vb;
-            p.e[m] = w2n;                    // workspace: the new w2 master, [M]
-        }
-    }
-    // the last CTA writes the served bf16 w2 (every CTA has read the forward's by now)
-    __threadfence();
-    __syncthreads();
-    if (t == 0) {
-        const uint32_t old = atomicAdd(p.ticket, 1u);
-        last = (old + 1u == gridDim.x * gridDim.y) ? 1 : 0;
-    }
+    if (t == 0) last = (ticket_old + 1u == gridDim.x * gridDim.y) ? 1 : 0;
     __syncthreads();
     if (!last) return;
     __threadfence();
