@@ -300,6 +300,13 @@ def time_vocab_shard(w, d, bk, bk_host, draft, P, stream, n=20):
             "note": "all-gathers not timed (one GPU)"}
 
 
+def hold_device(us: float):
+    """Keep the current stream busy for about `us` microseconds (a spin kernel), so that the
+    launches queued behind it run back to back on the device: timing a run of short kernels
+    this way measures the device, not the host's launch rate."""
+    torch.cuda._sleep(int(us * 2000))   # ~2 cycles per ns at the B200's 1.965 GHz clock
+
+
 def profile_head(w, dev, warmup, steps):
     """The length head and one online update of it at the workload's (B, H, M), no logits."""
     h, W1, b1, w2, b2 = (t.to(dev) if torch.is_tensor(t) else t for t in syn.make_head(w))
@@ -314,6 +321,7 @@ def profile_head(w, dev, warmup, steps):
     for name, fn in (("length_head_ms", lambda: api.svd_length_head(h, W1, b1, w2, b2, w.k, ws=ws)),
                      ("length_head_update_ms", lambda: trainer.step(h, label))):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        hold_device(60.0 * steps)
         e0.record()
         for _ in range(steps):
             fn()
@@ -500,6 +508,7 @@ def run_leg(w, args, info, dev, *, headline: bool, sweep=None):
         u0 = torch.cuda.Event(enable_timing=True)
         u1 = torch.cuda.Event(enable_timing=True)
         n_upd = 50
+        hold_device(60.0 * n_upd)   # the updates then run back to back on the device
         u0.record(stream)
         for _ in range(n_upd):
             trainer.step(d["h"], label)
