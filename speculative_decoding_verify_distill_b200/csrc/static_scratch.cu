@@ -27,7 +27,7 @@
 namespace {
 
 // Largest workspace the static scratch can stand in for: 4 MiB per device.  At k = 16 and a
-// 256-unit length head this covers batches of several hundred sequences (about 1.4 MiB at
+// 256-unit length head this covers batches of several hundred sequences (about 1.7 MiB at
 // B = 128); larger calls are rejected with SVD_ERR_WORKSPACE before anything is launched.
 constexpr size_t kScratchBytes = size_t(4) << 20;
 static_assert(kScratchBytes == SVD_NOALLOC_SCRATCH_BYTES, "header and library agree on the size");

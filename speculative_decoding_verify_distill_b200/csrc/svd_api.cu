@@ -67,7 +67,7 @@ HeadParams head_params(const uint16_t* h, const uint16_t* W1, const float* b1, c
     p.gamma = gamma; p.rnd = static_cast<int>(rnd);
     p.bhat = bhat_out; p.bk = bk_out; p.b2_dev = nullptr; p.u_out = nullptr;
     p.hdr = w.hdr; p.zpart = w.zpart; p.part = w.part; p.tile_ticket = w.tile_ticket;
-    p.nsplit = head_nsplit(B, M);
+    p.nsplit = head_nsplit(B, M, H);
     const int per = (H + p.nsplit - 1) / p.nsplit;
     p.ks = (per + 15) & ~15;
     return p;
@@ -284,7 +284,7 @@ svd_status svd_length_head_update(const svd_head_update_args* a, void* ws, size_
     hp.gamma = 1.f; hp.rnd = 0;
     hp.bhat = a->bhat; hp.bk = nullptr; hp.b2_dev = a->b2; hp.u_out = u;
     hp.hdr = w.hdr; hp.zpart = w.zpart; hp.part = w.part; hp.tile_ticket = w.tile_ticket;
-    hp.nsplit = head_nsplit(a->B, a->M);
+    hp.nsplit = head_nsplit(a->B, a->M, a->H);
     const int per = (a->H + hp.nsplit - 1) / hp.nsplit;
     hp.ks = (per + 15) & ~15;
     if (!have_fwd) {

@@ -33,11 +33,29 @@ constexpr int kHeadTileB = 16;   // sequences per length-head CTA
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // K splits of the length-head contraction: enough CTAs to cover the SMs twice over.
-__host__ __device__ inline int head_nsplit(int B, int M) {
+// K splits of the length head.  head_ws_splits: the splits the workspace holds partials for --
+// enough work units to fill the GPU (about two per SM) and, when the head has at most 32 output
+// tiles, at least 11, so that hidden sizes up to 11 x kHeadSplitCols columns split into pieces
+// the fused pass stages in one chunk of its large-vocabulary staging area (kHeadSplitCols
+// columns of 16 + 64 rows fit its 64 KB); at most kHeadMaxSplit.  head_nsplit: the splits a call
+// uses, within that.
+constexpr int kHeadMaxSplit = 16;
+constexpr int kHeadSplitCols = 400;
+__host__ __device__ inline int head_ws_splits(int B, int M) {
     if (B <= 0 || M <= 0) return 0;
     const int tiles = ((B + kHeadTileB - 1) / kHeadTileB) * ((M + kHeadTileM - 1) / kHeadTileM);
     int n = (296 + tiles - 1) / tiles;
-    return n < 1 ? 1 : (n > 16 ? 16 : n);
+    if (tiles <= 32 && n < 11) n = 11;
+    return n < 1 ? 1 : (n > kHeadMaxSplit ? kHeadMaxSplit : n);
+}
+__host__ __device__ inline int head_nsplit(int B, int M, int H) {
+    if (B <= 0 || M <= 0) return 0;
+    const int tiles = ((B + kHeadTileB - 1) / kHeadTileB) * ((M + kHeadTileM - 1) / kHeadTileM);
+    int n = (296 + tiles - 1) / tiles;
+    const int nk = (H + kHeadSplitCols - 1) / kHeadSplitCols;
+    if (nk > n) n = nk;
+    const int cap = head_ws_splits(B, M);
+    return n < 1 ? 1 : (n > cap ? cap : n);
 }
 
 struct WsLayout {
@@ -57,7 +75,7 @@ __host__ __device__ inline WsLayout ws_layout(int B, int k, int kt, int M) {
     L.zpart = off;
     off = align256(off + sizeof(float) * (size_t)mt * (size_t)B);
     L.part = off;
-    off = align256(off + sizeof(float) * (size_t)head_nsplit(B, M) * (size_t)B * (size_t)(M > 0 ? M : 0));
+    off = align256(off + sizeof(float) * (size_t)head_ws_splits(B, M) * (size_t)B * (size_t)(M > 0 ? M : 0));
     L.tile_ticket = off;   // output-tile tickets [bt * mt], then sequence-tile tickets [bt]
     off = align256(off + sizeof(uint32_t) * ((size_t)bt * (size_t)mt + (size_t)bt));
     // length-head update: pre-activations W1 h + b1 and backward terms, [B, M] fp32 each

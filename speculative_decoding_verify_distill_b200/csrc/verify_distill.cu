@@ -1205,6 +1205,9 @@ KernelFn pick_kernel(int flags, bool aligned) {
 // Vocabularies whose slices would need more than 16 CTAs take 256 x 10.
 constexpr int kSNT = 128, kSNV = 2, kSMB = 8;     //  2048 ids per CTA
 constexpr int kLNT = 256, kLNV = 8, kLMB = 3;     // 16384 ids per CTA
+// a length-head split of kHeadSplitCols columns stages in one chunk of this shape's staging area
+static_assert(((kLNV * kLNT * 32 / (2 * (kHeadTileB + kHeadTileM)) - 8) & ~15) >= kHeadSplitCols,
+              "head split width and staging area");
 constexpr int kXNT = 256, kXNV = 10, kXMB = 2;    // 20480 ids per CTA
 
 int next_pow2(int x) {
