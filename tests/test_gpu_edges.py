@@ -273,11 +273,14 @@ def test_empty_batch():
 
 
 @pytest.mark.parametrize("B,H,M,V", [(5, 272, 100, 20000), (17, 4096, 64, 16392),
-                                     (40, 1000, 300, 40960), (3, 16, 1, 151936)])
+                                     (40, 1000, 300, 40960), (3, 16, 1, 151936),
+                                     (40, 8192, 64, 40960), (9, 2048, 96, 8000)])
 def test_fused_head_ragged_shapes(B, H, M, V):
     """The length head inside the row pass on partial sequence / unit tiles (B % 16, M % 64 not
     zero), and the separate head kernel before it where H % 16 != 0: b_k, bhat and everything
-    downstream against the oracle."""
+    downstream against the oracle.  H = 8192 splits wider than one staging chunk of the row pass
+    (two chunks per unit), and V = 8000 takes the small-vocabulary shape, whose 8 KB staging area
+    holds 32 columns of a unit at a time."""
     k = 6
     g = torch.Generator().manual_seed(B * 7 + H + M)
     h = (3 * torch.randn((B, H), generator=g)).to(torch.bfloat16)
