@@ -288,7 +288,18 @@ def time_vocab_shard(w, d, bk, bk_host, draft, P, stream, n=20):
         ev[j][3].record(stream)
     torch.cuda.synchronize()
     part = [statistics.mean(ev[j][q].elapsed_time(ev[j][q + 1]) for j in range(n)) for q in range(3)]
-    rank_ms = statistics.mean(ev[j][0].elapsed_time(ev[j][3]) for j in range(n))
+    # the rank step as it runs: the calls back to back, no events between them (an event
+    # between two launches keeps the second from starting in the first one's tail)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hold_device(150.0 * n)
+    r0.record(stream)
+    for j in range(n):
+        s0.stats(stream)
+        s0.resolve(stream)
+        s0.finish(stream)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    rank_ms = r0.elapsed_time(r1) / n
     Vl = slices[0][1]
     alg = algorithmic_bytes(bk_host, w.k, w.kt, Vl)
     n1 = api.svd_vs_exchange_bytes(w.B, w.kt, 1)

@@ -40,6 +40,14 @@ constexpr int kVsUnroll = 4;                 // 16-byte vectors in flight per th
 constexpr uint32_t kNoId = 0xffffffffu;
 constexpr uint16_t kSentinel = 0xFF7Fu;      // lowest finite bf16: pads a ragged slice tail
 
+// Every kernel here is launched as a programmatic dependent of whatever precedes it on the
+// stream (launch_dependent below) and reads nothing before that grid has finished: the launch
+// latency overlaps the preceding kernel's tail (this rank's previous pass, or the all-gather).
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+
 __device__ __forceinline__ float neg_inf() { return -__int_as_float(0x7f800000); }
 __device__ __forceinline__ float quiet_nan() { return __int_as_float(0x7fc00000); }
 
@@ -118,6 +126,24 @@ struct VsParams {
     int32_t* n_emitted;
     svd_row_info* row_info;
 };
+
+// A programmatic dependent launch of one of the kernels below (see grid_dependency_wait).
+template <typename Kernel>
+cudaError_t launch_dependent(Kernel kernel, unsigned grid, unsigned block, cudaStream_t st,
+                             const VsParams& p) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(block, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 
 __device__ __forceinline__ int vs_bk(const VsParams& p, int b) {
     const int n = __ldg(p.bk + b);
@@ -248,6 +274,7 @@ template <bool ALIGNED>
 __global__ void __launch_bounds__(kVsThreads) vs_stats_kernel(const VsParams p) {
     __shared__ Partial redT[kVsWarps], redD[kVsWarps];
     __shared__ float sdm[kVsWarps];
+    grid_dependency_wait();
     const int row = blockIdx.x, t = threadIdx.x;
     const int b = row / p.kt, i = row % p.kt;
     const int n = vs_bk(p, b);
@@ -465,6 +492,7 @@ __device__ __forceinline__ svd_row_info row_info_of(const VsParams& p, const Row
 __global__ void __launch_bounds__(1024) vs_resolve_kernel(const VsParams p) {
     __shared__ RowState srow[33];
     __shared__ int bad;
+    grid_dependency_wait();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int b = blockIdx.x;
     const int k = p.k, kt = p.kt;
@@ -541,6 +569,7 @@ template <bool ALIGNED>
 __global__ void __launch_bounds__(kVsThreads) vs_masses_kernel(const VsParams p) {
     __shared__ float redf[kVsWarps];
     __shared__ unsigned long long redu[kVsWarps];
+    grid_dependency_wait();
     const int row = gridDim.x - 1 - blockIdx.x, t = threadIdx.x;   // reverse order, as finish
     const int b = row / p.kt, i = row % p.kt;
     const RowState s = p.rows[row];
@@ -654,6 +683,7 @@ template <bool ALIGNED, bool FP32>
 __global__ void __launch_bounds__(kVsThreads, 3) vs_finish_kernel(const VsParams p) {
     __shared__ unsigned long long scan[kVsWarps];
     __shared__ float part[kVsThreads];
+    grid_dependency_wait();
     __shared__ int found, last;
     const int row = gridDim.x - 1 - blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int b = row / p.kt, i = row % p.kt;
@@ -969,8 +999,9 @@ svd_status svd_vs_stats(const svd_vs_args* a, void* send1, void* ws, size_t ws_b
     p.send1 = static_cast<Rec1*>(send1);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const unsigned grid = static_cast<unsigned>(a->B) * a->kt;
-    if (slice_aligned(a, false)) vs_stats_kernel<true><<<grid, kVsThreads, 0, st>>>(p);
-    else vs_stats_kernel<false><<<grid, kVsThreads, 0, st>>>(p);
+    const cudaError_t err = slice_aligned(a, false) ? launch_dependent(vs_stats_kernel<true>, grid, kVsThreads, st, p)
+                                                    : launch_dependent(vs_stats_kernel<false>, grid, kVsThreads, st, p);
+    if (err != cudaSuccess) return SVD_ERR_CUDA;
     return launched();
 }
 
@@ -985,12 +1016,15 @@ svd_status svd_vs_resolve(const svd_vs_args* a, const void* recv1, void* send2, 
     p.recv1 = static_cast<const Rec1*>(recv1);
     p.send2 = static_cast<Rec2*>(send2);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    vs_resolve_kernel<<<a->B, 32 * (a->kt < 32 ? a->kt : 32), 0, st>>>(p);
+    if (launch_dependent(vs_resolve_kernel, static_cast<unsigned>(a->B), 32u * (a->kt < 32 ? a->kt : 32), st, p) !=
+        cudaSuccess)
+        return SVD_ERR_CUDA;
     s = launched();
     if (s != SVD_OK) return s;
     const unsigned grid = static_cast<unsigned>(a->B) * a->kt;
-    if (slice_aligned(a, false)) vs_masses_kernel<true><<<grid, kVsThreads, 0, st>>>(p);
-    else vs_masses_kernel<false><<<grid, kVsThreads, 0, st>>>(p);
+    const cudaError_t err = slice_aligned(a, false) ? launch_dependent(vs_masses_kernel<true>, grid, kVsThreads, st, p)
+                                                    : launch_dependent(vs_masses_kernel<false>, grid, kVsThreads, st, p);
+    if (err != cudaSuccess) return SVD_ERR_CUDA;
     return launched();
 }
 
@@ -1007,10 +1041,11 @@ svd_status svd_vs_finish(const svd_vs_args* a, const void* recv2, void* ws, size
     const unsigned grid = static_cast<unsigned>(a->B) * a->kt;
     const bool al = slice_aligned(a, a->distill != 0);
     const bool f32 = a->distill && a->dlogits_fp32;
-    if (al && f32) vs_finish_kernel<true, true><<<grid, kVsThreads, 0, st>>>(p);
-    else if (al) vs_finish_kernel<true, false><<<grid, kVsThreads, 0, st>>>(p);
-    else if (f32) vs_finish_kernel<false, true><<<grid, kVsThreads, 0, st>>>(p);
-    else vs_finish_kernel<false, false><<<grid, kVsThreads, 0, st>>>(p);
+    const cudaError_t err = (al && f32) ? launch_dependent(vs_finish_kernel<true, true>, grid, kVsThreads, st, p)
+                            : al        ? launch_dependent(vs_finish_kernel<true, false>, grid, kVsThreads, st, p)
+                            : f32       ? launch_dependent(vs_finish_kernel<false, true>, grid, kVsThreads, st, p)
+                                        : launch_dependent(vs_finish_kernel<false, false>, grid, kVsThreads, st, p);
+    if (err != cudaSuccess) return SVD_ERR_CUDA;
     return launched();
 }
 

@@ -64,8 +64,12 @@ def _check_step(tr, h, label, step):
     return ref
 
 
-@pytest.mark.parametrize("B,H,M", [(32, 512, 64), (7, 300, 37), (128, 4096, 256)])
+@pytest.mark.parametrize("B,H,M", [(32, 512, 64), (7, 300, 37), (128, 4096, 256), (200, 1024, 128),
+                                   (300, 520, 70)])
 def test_update_steps_match_oracle(B, H, M):
+    """Three AdamW steps against the oracle.  B = 200 and 300 take the backward through more than
+    one 128-sequence chunk (the later chunks staged after the first); H = 520 and M = 70 leave
+    partial 64-column and 64-unit blocks (plain loads where a staged row would run past H or M)."""
     w = syn.WORKLOADS["ragged_qwen_b128"].with_(B=B, H=H, M=M)
     h, W1, b1, w2, b2 = syn.make_head(w)
     tr = api.LengthHeadTrainer(W1.cuda(), b1.cuda(), w2.cuda(), b2, B, lr=LR)
