@@ -295,18 +295,24 @@ __global__ void __launch_bounds__(kVsThreads) vs_stats_kernel(const VsParams p) 
     const int nvec = (p.Vl + 7) >> 3;
     Partial aT{neg_inf(), 0.f, 0.f, kNoId}, aD{neg_inf(), 0.f, 0.f, kNoId};
     float dmax = neg_inf();
-    for (int g0 = t; g0 < nvec; g0 += kVsThreads * kVsUnroll) {
-        uint4 tv[kVsUnroll], dv[kVsUnroll];
+    // The thread's vectors g = t, t + 256, ... in order, two at a time, with the next two
+    // already loading while these are absorbed (two register buffers, A and B, in turn).
+    constexpr int kG = kVsUnroll / 2;
+    constexpr int kStep = kVsThreads * kG;
+    uint4 tA[kG], dA[kG], tB[kG], dB[kG];
+    auto load_group = [&](uint4 (&tv)[kG], uint4 (&dv)[kG], int g0) {
 #pragma unroll
-        for (int u = 0; u < kVsUnroll; ++u) {
+        for (int u = 0; u < kG; ++u) {
             const int g = g0 + u * kVsThreads;
             if (g < nvec) {
                 tv[u] = load_vec<ALIGNED>(Trow, g, p.Vl);
                 if (verified) dv[u] = load_vec<ALIGNED>(Drow, g, p.Vl);
             }
         }
+    };
+    auto absorb_group = [&](const uint4 (&tv)[kG], const uint4 (&dv)[kG], int g0) {
 #pragma unroll
-        for (int u = 0; u < kVsUnroll; ++u) {
+        for (int u = 0; u < kG; ++u) {
             const int g = g0 + u * kVsThreads;
             if (g >= nvec) break;
             absorb(aT, tv[u], g, p.k2, exps, nullptr, nullptr);
@@ -316,6 +322,17 @@ __global__ void __launch_bounds__(kVsThreads) vs_stats_kernel(const VsParams p) 
                 absorb(aD, dv[u], g, p.k2, exps, &xt, &dmax);
             }
         }
+    };
+    int g0 = t;
+    if (g0 < nvec) load_group(tA, dA, g0);
+    while (g0 < nvec) {
+        if (g0 + kStep < nvec) load_group(tB, dB, g0 + kStep);
+        absorb_group(tA, dA, g0);
+        g0 += kStep;
+        if (g0 >= nvec) break;
+        if (g0 + kStep < nvec) load_group(tA, dA, g0 + kStep);
+        absorb_group(tB, dB, g0);
+        g0 += kStep;
     }
     const Partial cT = combine_block(aT, p.k2, exps, redT);
     Partial cD{neg_inf(), 0.f, 0.f, kNoId};
@@ -724,18 +741,24 @@ __global__ void __launch_bounds__(kVsThreads, 3) vs_finish_kernel(const VsParams
                 if (p.row_info) p.row_info[row].loss = L;
             }
             const int yl = s.y - p.v0;    // the target argmax, if this slice holds it
-            for (int g0 = t; g0 < nvec; g0 += kVsThreads * kVsUnroll) {
-                uint4 tv[kVsUnroll], dv[kVsUnroll];
+            // the thread's vectors two at a time, the next two loading while these are written
+            // (register buffers A and B in turn)
+            constexpr int kG = kVsUnroll / 2;
+            constexpr int kStep = kVsThreads * kG;
+            uint4 tA[kG], dA[kG], tB[kG], dB[kG];
+            auto load_group = [&](uint4 (&tv)[kG], uint4 (&dv)[kG], int g0) {
 #pragma unroll
-                for (int u = 0; u < kVsUnroll; ++u) {
+                for (int u = 0; u < kG; ++u) {
                     const int g = g0 + u * kVsThreads;
                     if (g < nvec) {
                         tv[u] = load_vec<ALIGNED>(Trow, g, p.Vl);
                         dv[u] = load_vec<ALIGNED>(Drow, g, p.Vl);
                     }
                 }
+            };
+            auto grad_group = [&](const uint4 (&tv)[kG], const uint4 (&dv)[kG], int g0) {
 #pragma unroll
-                for (int u = 0; u < kVsUnroll; ++u) {
+                for (int u = 0; u < kG; ++u) {
                     const int g = g0 + u * kVsThreads;
                     if (g >= nvec) break;
                     float xt[8], xd[8], gl[8];
@@ -764,6 +787,17 @@ __global__ void __launch_bounds__(kVsThreads, 3) vs_finish_kernel(const VsParams
                     }
                     store_grad<ALIGNED, FP32>(p, drow, g, gl);
                 }
+            };
+            int g0 = t;
+            if (g0 < nvec) load_group(tA, dA, g0);
+            while (g0 < nvec) {
+                if (g0 + kStep < nvec) load_group(tB, dB, g0 + kStep);
+                grad_group(tA, dA, g0);
+                g0 += kStep;
+                if (g0 >= nvec) break;
+                if (g0 + kStep < nvec) load_group(tA, dA, g0 + kStep);
+                grad_group(tB, dB, g0);
+                g0 += kStep;
             }
         } else {
             // rows past b_k (and the bonus row's draft slot): zero gradient, zero loss
