@@ -11,8 +11,11 @@
 //      residual falls back to p without a second pass), sent to every CTA of the cluster over
 //      distributed shared memory;
 //   2. every CTA forms the same totals and the same prefix in rank order; the CTA whose
-//      interval holds the target floor(R * u / 2^24) searches its slice in rounds of 256
-//      vectors with a block scan and writes the token.
+//      interval holds the target floor(R * u / 2^24) finds the round of 256 vectors that holds
+//      it from the per-round masses it kept in shared memory in step 1, the vector by a block
+//      scan over that round, and the token by re-reading that one vector.  (Slices of more
+//      than 16 rounds, and an empty residual that falls back to p, search by re-reading the
+//      slice round by round instead.)
 // Integer masses make the prefix sums exact and associative, so the split over CTAs cannot
 // change the draw.  Element arithmetic is the row pass's (svd_device.cuh) with lse(D/tau) and
 // lse(T/tau) read back from the row record.
@@ -27,6 +30,8 @@ constexpr int kFixThreads = 256;
 constexpr int kFixWarps = kFixThreads / 32;
 constexpr int kFixMaxCluster = 8;
 constexpr int kFixSlice = 16384;              // ids per CTA before the cluster grows
+constexpr int kFixMaxRounds = 16;             // rounds of 256 vectors whose masses are kept
+constexpr int kFixUnroll = 2;                 // vectors in flight per thread in step 1
 
 // Vector g (ids 8g .. 8g+7) of a row of V ids; ids past V read as the lowest finite bf16,
 // whose probability is 0.
@@ -65,11 +70,14 @@ __device__ __forceinline__ void vec_masses(const uint4& tv, const uint4& dv, boo
 }
 
 template <bool ALIGNED>
-__global__ void __launch_bounds__(kFixThreads) sample_fix_kernel(const RowParams p, int slice) {
+__global__ void __launch_bounds__(kFixThreads, 4) sample_fix_kernel(const RowParams p, int slice) {
     __shared__ unsigned long long red[2][kFixWarps];
     __shared__ unsigned long long cm[kFixMaxCluster][2];   // [rank][residual, p] masses
     __shared__ unsigned long long scan[kFixWarps];
-    __shared__ int found;
+    __shared__ unsigned long long vmr[kFixMaxRounds][kFixThreads];   // [round][thread] masses
+    __shared__ unsigned long long rtot[kFixMaxRounds][kFixWarps];    // [round][warp] sums
+    __shared__ int found, sround;
+    __shared__ unsigned long long srel;
     // launched as a programmatic dependent of the finalize pass: wait for its accepted lengths
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -92,15 +100,37 @@ __global__ void __launch_bounds__(kFixThreads) sample_fix_kernel(const RowParams
     const int v1 = min(V, v0 + slice);
     const int gbeg = v0 / 8, gend = v1 > v0 ? (v1 + 7) / 8 : gbeg;
 
-    // 1. this slice's masses, to every CTA of the cluster
+    // 1. this slice's masses, to every CTA of the cluster; per round of 256 vectors each thread
+    //    also keeps its vector's mass of the column a search would use (residual, or p)
+    const int rounds = (gend - gbeg + kFixThreads - 1) / kFixThreads;
+    const bool keep = rounds <= kFixMaxRounds;
     unsigned long long m = 0ull, pm = 0ull;
-    for (int g = gbeg + t; g < gend; g += kFixThreads) {
-        const uint4 tv = row_vec<ALIGNED>(Trow, g, V);
-        const uint4 dv = residual ? row_vec<ALIGNED>(Drow, g, V) : tv;
-        unsigned long long wp[8], wr[8];
-        vec_masses(tv, dv, residual, k2, L2T, L2D, wp, wr);
+    for (int i0 = 0; i0 < rounds; i0 += kFixUnroll) {
+        uint4 tv[kFixUnroll], dv[kFixUnroll];
 #pragma unroll
-        for (int l = 0; l < 8; ++l) { m += wr[l]; pm += wp[l]; }
+        for (int u = 0; u < kFixUnroll; ++u) {
+            const int g = gbeg + t + (i0 + u) * kFixThreads;
+            if (g < gend) {
+                tv[u] = row_vec<ALIGNED>(Trow, g, V);
+                dv[u] = residual ? row_vec<ALIGNED>(Drow, g, V) : tv[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kFixUnroll; ++u) {
+            const int i = i0 + u;
+            if (i >= rounds) break;
+            const int g = gbeg + t + i * kFixThreads;
+            unsigned long long vr = 0ull, vp = 0ull;
+            if (g < gend) {
+                unsigned long long wp[8], wr[8];
+                vec_masses(tv[u], dv[u], residual, k2, L2T, L2D, wp, wr);
+#pragma unroll
+                for (int l = 0; l < 8; ++l) { vr += wr[l]; vp += wp[l]; }
+            }
+            m += vr;
+            pm += vp;
+            if (keep) vmr[i][t] = residual ? vr : vp;
+        }
     }
     m = warp_sum_u64(m);
     pm = warp_sum_u64(pm);
@@ -134,6 +164,67 @@ __global__ void __launch_bounds__(kFixThreads) sample_fix_kernel(const RowParams
     const unsigned long long rel = tgt - before;
     const bool res = residual && col == 0;
     if (t == 0) found = -1;
+    if (keep && col == 0) {
+        // the round holding the target, from the kept masses (every thread of a round holds the
+        // vector gbeg + t + i * 256, so thread order is id order within a round)
+        for (int i = 0; i < rounds; ++i) {
+            const unsigned long long ws = warp_sum_u64(vmr[i][t]);
+            if (lane == 0) rtot[i][warp] = ws;
+        }
+        __syncthreads();
+        if (t == 0) {
+            unsigned long long run = 0ull;
+            sround = rounds - 1;
+            srel = 0ull;
+            for (int i = 0; i < rounds; ++i) {
+                unsigned long long tot = 0ull;
+                for (int q = 0; q < kFixWarps; ++q) tot += rtot[i][q];
+                if (rel - run < tot) {   // run <= rel throughout: the first round passing rel
+                    sround = i;
+                    srel = rel - run;
+                    break;
+                }
+                run += tot;
+            }
+        }
+        __syncthreads();
+        const int i = sround;
+        const unsigned long long rr = srel;
+        const unsigned long long vm = vmr[i][t];
+        unsigned long long incl = vm;
+        warp_inclusive_scan_u64(incl);
+        if (lane == 31) scan[warp] = incl;
+        __syncthreads();
+        unsigned long long wbefore = 0ull;
+#pragma unroll
+        for (int q = 0; q < kFixWarps; ++q)
+            if (q < warp) wbefore += scan[q];
+        const unsigned long long lo = wbefore + incl - vm;
+        if (vm > 0ull && lo <= rr && rr - lo < vm) {
+            // the target lies in this vector: its 8 masses again, walked in id order
+            const int g = gbeg + t + i * kFixThreads;
+            const uint4 tv = row_vec<ALIGNED>(Trow, g, V);
+            const uint4 dv = res ? row_vec<ALIGNED>(Drow, g, V) : tv;
+            unsigned long long w[8], wr[8];
+            vec_masses(tv, dv, res, k2, L2T, L2D, w, wr);
+            const unsigned long long r8 = rr - lo;
+            unsigned long long cum = 0ull;
+            int pick = -1;
+#pragma unroll
+            for (int l = 0; l < 8; ++l) {
+                cum += res ? wr[l] : w[l];
+                if (pick < 0 && cum > r8) pick = l;
+            }
+            found = g * 8 + (pick < 0 ? 7 : pick);
+        }
+        __syncthreads();
+        if (t == 0 && found >= 0) {
+            p.emitted[static_cast<size_t>(b) * (k + 1) + a] = found;
+            p.rec[static_cast<size_t>(b) * kt + fix].sample_token = found;
+            if (p.row_info) p.row_info[static_cast<size_t>(b) * kt + fix].sample_token = found;
+        }
+        return;
+    }
     unsigned long long run = 0ull;    // mass of this slice's vectors before the round, id order
     for (int r0 = gbeg; r0 < gend; r0 += kFixThreads) {
         const int g = r0 + t;
